@@ -1,0 +1,333 @@
+"""HARP rotation oracle: a plain, slow, float64 CPU restatement of the transform.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code with
+the CUDA library (no kernels, headers, tables or helpers) and never calls it.
+
+What it computes (sources are the HARP pages: "Technical Summary: HARP
+(Hadamard-Preconditioned Adaptive Rotation Processor)", gist.science, and its
+Chinese twin; the arXiv abstract "HARP: Hadamard-Preconditioned Adaptive
+Rotation Processor for Extreme LLM Quantization"):
+
+* §2.1 Core Architecture: a mixed-radix schedule b = (b_0..b_{m-1}) with
+  prod b_t = d; stage t applies a block-diagonal orthogonal matrix to groups of
+  b_t coordinates separated by stride permutations.
+* §2.2 Hadamard Preconditioning: every block is B_{t,c}(theta) = Q_{t,c}(theta) G_{b_t};
+  G is the normalized Sylvester Hadamard for powers of two, else the QR of a fixed
+  Gaussian matrix; Q is a Givens rotation for b=2 and a Cayley map for b>2;
+  theta = 0 gives Q = I and the fixed randomized Hadamard transform.
+* §2.4 Deployment Efficiency: theta may be stored as int8.
+* Abstract: a two-sided processor (one rotation on each side of a weight).
+
+Readings taken where the pages leave a step open (each is also listed in the
+design notes):
+
+* digit order: index i = sum_t i_t s_t with s_t = prod_{j<t} b_j (digit 0 least
+  significant); stage t mixes digit t; block index c = lo + s_t*hi with
+  lo = i mod s_t, hi = i div (s_t b_t).
+* order: y = M_{m-1} ... M_1 M_0 S x (random signs first, stage 0 next).
+* S: s_i = -1 if the top bit of the i-th SplitMix64 output of the sign seed is
+  set, else +1.
+* G_b (b not a power of two): one matrix per radix value; entries row-major from
+  a SplitMix64 stream seeded with (qr_seed or 0x4841525000000000) + b; each
+  entry consumes two outputs u1, u2 mapped to U = (u >> 11) 2^-53 and
+  g = sqrt(-2 ln(1-U1)) cos(2 pi U2); G = Q diag(sign R_kk) from M = QR, sign(0)=+1.
+* G_b (power of two): G[k][l] = (-1)^popcount(k & l) / sqrt(b).
+* Givens: Q(theta) = [[cos, -sin], [sin, cos]].
+* Cayley: A[i][j] = theta_k for i<j in row-major order of the strict upper
+  triangle, A[j][i] = -theta_k, Q = (I - A)^{-1} (I + A); one parameter set per block.
+* theta layout: stages in order; within a stage, blocks in c order; p_t
+  parameters per block (1 for b=2, b(b-1)/2 otherwise).
+* int8 theta: theta = q * scale_t, one float32 scale per stage.
+* two-sided: W_out = T_U^T W T_V (rows of W take the inverse V transform, columns
+  the inverse U transform).
+
+Pins (tests/test_oracle_pins.py): SplitMix64 published outputs, Gaussian
+statistics, scipy's Sylvester Hadamard, the unique positive-diagonal QR, Givens
+group law, Cayley orthogonality / det +1 / closed forms, theta=0 Kronecker form,
+an independent tensor-axis restatement of the stages, dense orthogonality,
+round trips and bf16 rounding of hand-worked values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional, Sequence
+
+import numpy as np
+import scipy.sparse as sp
+
+MASK64 = (1 << 64) - 1
+GOLDEN_GAMMA = 0x9E3779B97F4A7C15
+QR_SEED_BASE = 0x4841525000000000  # "HARP" in the top four bytes
+
+
+# ---------------------------------------------------------------------------
+# SplitMix64 (Steele, Lea & Flood, "Fast splittable pseudorandom number
+# generators", OOPSLA 2014; the 64-bit finalizer of Vigna's reference code)
+# ---------------------------------------------------------------------------
+
+def splitmix64(seed: int, n: int) -> List[int]:
+    """The first n outputs of the SplitMix64 stream whose state starts at seed."""
+    state = seed & MASK64
+    out = []
+    for _ in range(n):
+        state = (state + GOLDEN_GAMMA) & MASK64
+        z = state
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64
+        out.append(z ^ (z >> 31))
+    return out
+
+
+def unit_double(u: int) -> float:
+    """Top 53 bits of a 64-bit output as a double in [0, 1)."""
+    return (u >> 11) * 2.0 ** -53
+
+
+def sign_vector(d: int, sign_seed: int) -> np.ndarray:
+    """The random +-1 diagonal S of the randomized Hadamard transform."""
+    return np.array([-1.0 if (u >> 63) else 1.0 for u in splitmix64(sign_seed, d)])
+
+
+def gaussian_matrix(b: int, seed: int) -> np.ndarray:
+    """b x b standard normal entries, row-major, Box-Muller cosine branch."""
+    u = splitmix64(seed, 2 * b * b)
+    g = np.empty(b * b)
+    for e in range(b * b):
+        u1 = unit_double(u[2 * e])
+        u2 = unit_double(u[2 * e + 1])
+        g[e] = math.sqrt(-2.0 * math.log(1.0 - u1)) * math.cos(2.0 * math.pi * u2)
+    return g.reshape(b, b)
+
+
+# ---------------------------------------------------------------------------
+# Base mixers G_b (§2.2 "G_{b_t} is a fixed base mixer")
+# ---------------------------------------------------------------------------
+
+def is_pow2(b: int) -> bool:
+    return b >= 1 and (b & (b - 1)) == 0
+
+
+def sylvester_mixer(b: int) -> np.ndarray:
+    """Normalized Sylvester Hadamard: entry (k, l) is (-1)^popcount(k & l) / sqrt(b)."""
+    g = np.empty((b, b))
+    for k in range(b):
+        for l in range(b):
+            g[k, l] = -1.0 if bin(k & l).count("1") % 2 else 1.0
+    return g / math.sqrt(b)
+
+
+def qr_mixer(b: int, qr_seed: int = 0) -> np.ndarray:
+    """Deterministic orthogonal fallback: Q factor of a fixed seeded Gaussian
+    matrix, columns signed so that R has a non-negative diagonal."""
+    base = qr_seed if qr_seed else QR_SEED_BASE
+    m = gaussian_matrix(b, (base + b) & MASK64)
+    q, r = np.linalg.qr(m)
+    sgn = np.where(np.diag(r) < 0, -1.0, 1.0)
+    return q * sgn[None, :]
+
+
+def base_mixer(b: int, qr_seed: int = 0) -> np.ndarray:
+    return sylvester_mixer(b) if is_pow2(b) else qr_mixer(b, qr_seed)
+
+
+# ---------------------------------------------------------------------------
+# Learnable factor Q_{t,c}(theta) (§2.2)
+# ---------------------------------------------------------------------------
+
+def params_per_block(b: int) -> int:
+    return 1 if b == 2 else b * (b - 1) // 2
+
+
+def givens(theta: float) -> np.ndarray:
+    c, s = math.cos(theta), math.sin(theta)
+    return np.array([[c, -s], [s, c]])
+
+
+def skew_from_params(params: Sequence[float], b: int) -> np.ndarray:
+    a = np.zeros((b, b))
+    k = 0
+    for i in range(b):
+        for j in range(i + 1, b):
+            a[i, j] = params[k]
+            a[j, i] = -params[k]
+            k += 1
+    return a
+
+
+def cayley(params: Sequence[float], b: int) -> np.ndarray:
+    a = skew_from_params(params, b)
+    eye = np.eye(b)
+    return np.linalg.solve(eye - a, eye + a)
+
+
+def learnable_factor(params: Sequence[float], b: int) -> np.ndarray:
+    if b == 2:
+        return givens(float(params[0]))
+    return cayley(params, b)
+
+
+# ---------------------------------------------------------------------------
+# Plan: schedule, strides, theta layout
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class OraclePlan:
+    d: int
+    schedule: tuple
+    theta: np.ndarray                 # float64, concatenated per stage/block
+    sign_seed: int
+    qr_seed: int = 0
+
+    def __post_init__(self):
+        self.schedule = tuple(int(b) for b in self.schedule)
+        if int(np.prod(self.schedule)) != self.d:
+            raise ValueError("product of the schedule must equal d")
+        self.theta = np.asarray(self.theta, dtype=np.float64)
+        if self.theta.size != theta_count(self.schedule):
+            raise ValueError("theta has the wrong length for this schedule")
+
+    @property
+    def m(self) -> int:
+        return len(self.schedule)
+
+
+def strides(schedule: Sequence[int]) -> List[int]:
+    s, out = 1, []
+    for b in schedule:
+        out.append(s)
+        s *= b
+    return out
+
+
+def stage_theta_counts(schedule: Sequence[int]) -> List[int]:
+    d = int(np.prod(schedule))
+    return [(d // b) * params_per_block(b) for b in schedule]
+
+
+def theta_count(schedule: Sequence[int]) -> int:
+    return sum(stage_theta_counts(schedule))
+
+
+def dequantize_int8(codes: np.ndarray, scales: np.ndarray, schedule: Sequence[int]) -> np.ndarray:
+    """int8 storage (§2.4): theta = q * scale_t in float64."""
+    out = np.empty(codes.size)
+    off = 0
+    for t, n in enumerate(stage_theta_counts(schedule)):
+        out[off:off + n] = codes[off:off + n].astype(np.float64) * float(scales[t])
+        off += n
+    return out
+
+
+def make_plan(d, schedule, theta=None, sign_seed=0, qr_seed=0, codes=None, scales=None) -> OraclePlan:
+    if codes is not None:
+        theta = dequantize_int8(np.asarray(codes), np.asarray(scales), schedule)
+    if theta is None:
+        theta = np.zeros(theta_count(schedule))
+    return OraclePlan(int(d), tuple(schedule), np.asarray(theta, dtype=np.float64),
+                      int(sign_seed), int(qr_seed))
+
+
+# ---------------------------------------------------------------------------
+# Blocks B_{t,c} = Q_{t,c}(theta) G_{b_t} and explicit sparse stage matrices
+# ---------------------------------------------------------------------------
+
+def stage_blocks(plan: OraclePlan) -> List[np.ndarray]:
+    """Per stage, an array [d/b_t, b_t, b_t] holding B_{t,c}[k][l] (k out, l in)."""
+    blocks = []
+    off = 0
+    for b in plan.schedule:
+        g = base_mixer(b, plan.qr_seed)
+        p = params_per_block(b)
+        nb = plan.d // b
+        bt = np.empty((nb, b, b))
+        for c in range(nb):
+            q = learnable_factor(plan.theta[off + c * p: off + (c + 1) * p], b)
+            bt[c] = q @ g
+        off += nb * p
+        blocks.append(bt)
+    return blocks
+
+
+def stage_matrix(d: int, b: int, s: int, blocks_t: np.ndarray) -> sp.csr_matrix:
+    """M_t with M_t[lo + s(k + b hi), lo + s(l + b hi)] = B_{t,c}[k][l], c = lo + s hi."""
+    rows, cols, vals = [], [], []
+    for c in range(d // b):
+        lo, hi = c % s, c // s
+        for k in range(b):
+            for l in range(b):
+                rows.append(lo + s * (k + b * hi))
+                cols.append(lo + s * (l + b * hi))
+                vals.append(blocks_t[c, k, l])
+    return sp.csr_matrix((vals, (rows, cols)), shape=(d, d))
+
+
+def stage_matrices(plan: OraclePlan) -> List[sp.csr_matrix]:
+    blocks = stage_blocks(plan)
+    return [stage_matrix(plan.d, b, s, blocks[t])
+            for t, (b, s) in enumerate(zip(plan.schedule, strides(plan.schedule)))]
+
+
+class Transform:
+    """T = M_{m-1} ... M_0 S for one plan, with its stage matrices built once."""
+
+    def __init__(self, plan: OraclePlan):
+        self.plan = plan
+        self.signs = sign_vector(plan.d, plan.sign_seed)
+        self.mats = stage_matrices(plan)
+
+    def forward(self, x: np.ndarray) -> np.ndarray:
+        """y = T x for every row x of a [rows, d] array."""
+        z = np.asarray(x, dtype=np.float64) * self.signs[None, :]
+        for mt in self.mats:
+            z = (mt @ z.T).T
+        return z
+
+    def inverse(self, y: np.ndarray) -> np.ndarray:
+        """x = T^T y = S M_0^T ... M_{m-1}^T y for every row."""
+        z = np.asarray(y, dtype=np.float64)
+        for mt in reversed(self.mats):
+            z = (mt.T @ z.T).T
+        return z * self.signs[None, :]
+
+    def apply(self, x: np.ndarray, direction: str) -> np.ndarray:
+        if direction == "forward":
+            return self.forward(x)
+        if direction == "inverse":
+            return self.inverse(x)
+        raise ValueError(direction)
+
+    def dense(self) -> np.ndarray:
+        """T itself, built column by column from the unit vectors."""
+        return self.forward(np.eye(self.plan.d)).T
+
+
+def apply(plan: OraclePlan, x: np.ndarray, direction: str = "forward") -> np.ndarray:
+    return Transform(plan).apply(x, direction)
+
+
+def two_sided(plan_u: OraclePlan, plan_v: OraclePlan, w: np.ndarray) -> np.ndarray:
+    """W_out = T_U^T W T_V for W of shape [d_U, d_V] (abstract: two-sided processor)."""
+    tv = Transform(plan_v)
+    tu = Transform(plan_u)
+    z = tv.inverse(np.asarray(w, dtype=np.float64))      # rows: w_r^T T_V = (T_V^T w_r)^T
+    return tu.inverse(z.T).T                             # columns: T_U^T col
+
+
+# ---------------------------------------------------------------------------
+# Output rounding to the I/O dtype
+# ---------------------------------------------------------------------------
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bf16 value (8 significant bits, ties to even) of each float64,
+    rounded directly from float64; returned as float64."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m 2^e, 0.5 <= |m| < 1
+    normal = np.ldexp(np.rint(m * 256.0), e - 8)
+    sub = np.rint(x * 2.0 ** 133) * 2.0 ** -133   # below 2^-126: fixed spacing 2^-133
+    return np.where(np.abs(x) < 2.0 ** -126, sub, normal)
+
+
+def round_f32(x: np.ndarray) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
