@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the HARP rotation hot path on B200.
+
+One step = one harp_apply (forward) over a batch of the d=4096, schedule
+(8,8,8,8) workload: 65,536 bf16 rows per GPU (Student-t nu=3 entries, 8 outlier
+channels x50, theta ~ N(0, 0.05)), inputs already resident in HBM.  The batch is
+512 MiB in and 512 MiB out, larger than L2 (126 MB), so no flush is needed
+between steps.  With N GPUs (one process per GPU, launched by torchrun) every rank
+rotates its own 65,536-row shard (weak scaling, no data-path collective).
+
+Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU oracle on
+a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HARP rotation rows/s and HBM GB/s (fraction of B200 roofline), d=4096/5120/8192"
+UNIT = "rows/s"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD_TEXT = {
+    "c2": "d=4096 schedule (8,8,8,8), 65536 rows/GPU bf16 Student-t(3) with 8 outlier channels x50, "
+          "theta~N(0,0.05), forward",
+    "c3_64k": "d=5120 schedule (8,8,8,5,2), 65536 rows/GPU bf16 N(0,1) with 1% entries x20, forward",
+    "c5": "d=8192 schedule (8,8,8,8,2), int8 theta + per-stage scale, 65536 rows/GPU bf16 N(0,1), forward",
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--no-extra", action="store_true", help="skip the d=5120 / d=8192 side measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="harp_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[1]), "max": float(parts[2]), "util": float(parts[4]),
+                                 "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pcap": parts[9]})
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        load = [r for r in rows if r["util"] >= 50] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# --------------------------------------------------------------- profiles ---
+
+def kernel_sources():
+    d = os.path.join(ROOT, "structured_rotations_b200", "csrc")
+    return {f: os.path.join(d, f) for f in os.listdir(d)}
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel source
+    hash still matches the source being benchmarked; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_src = re.search(r"^source_file:\s*(\S+)", text, re.M)
+    m_sha = re.search(r"^source_sha256:\s*([0-9a-f]{64})", text, re.M)
+    m_b = re.search(r"^dram_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    if not (m_src and m_sha and m_b):
+        return None
+    src = kernel_sources().get(m_src.group(1))
+    if not src:
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return float(m_b.group(1)) if sha == m_sha.group(1) else None
+
+
+# ------------------------------------------------------------- workloads ---
+
+def make_plan(name, H, W, O_theta_count=None):
+    w = W.get(name)
+    n = H.theta_count(w.schedule)
+    theta = W.draw_theta(n, w.theta_sigma, w.theta_seed)
+    if w.theta_kind == "i8":
+        counts = [(w.d // b) * (1 if b == 2 else b * (b - 1) // 2) for b in w.schedule]
+        codes, scales = W.quantize_theta_int8(theta, counts)
+        return H.Plan(w.d, w.schedule, codes=codes, scales=scales, sign_seed=w.sign_seed).materialize()
+    return H.Plan(w.d, w.schedule, theta=theta, sign_seed=w.sign_seed).materialize()
+
+
+def to_device_bf16(enc, torch, device):
+    import numpy as np
+    return torch.from_numpy(enc.view(np.int16)).view(torch.bfloat16).to(device)
+
+
+# ------------------------------------------------------------- reference ---
+
+def run_reference(args):
+    import numpy as np
+    import workloads as W
+    from oracle import harp_oracle as O
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.get(args.workload)
+    theta = W.draw_theta(O.theta_count(w.schedule), w.theta_sigma, w.theta_seed)
+    if w.theta_kind == "i8":
+        codes, scales = W.quantize_theta_int8(theta, O.stage_theta_counts(w.schedule))
+        plan = O.make_plan(w.d, w.schedule, codes=codes, scales=scales, sign_seed=w.sign_seed)
+    else:
+        plan = O.make_plan(w.d, w.schedule, theta, sign_seed=w.sign_seed)
+    tr = O.Transform(plan)
+    sample = 256
+    x = W.draw_rows(w, 0, sample)
+    for _ in range(args.warmup):
+        tr.forward(x)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        tr.forward(x)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = sample * args.steps / total
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "rows_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{sample} rows of the workload per step (float64 scipy CSR stages, one core)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def cpu_baseline(args, W):
+    from oracle import harp_oracle as O
+    w = W.get(args.workload)
+    theta = W.draw_theta(O.theta_count(w.schedule), w.theta_sigma, w.theta_seed)
+    tr = O.Transform(O.make_plan(w.d, w.schedule, theta, sign_seed=w.sign_seed))
+    chunk = 512
+    x = W.draw_rows(w, 0, chunk)
+    rows, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < args.cpu_seconds:
+        tr.forward(x)
+        rows += chunk
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{rows} rows of the workload ({chunk}-row chunks, float64 scipy CSR stages, "
+                      f"one core) in {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ ours ---
+
+def time_apply(plan, x, y, steps, warmup, torch, dist=None):
+    """Warm up, then time exactly `steps` applies between a barrier and a sync on
+    both sides.  Returns (elapsed_ms, mean kernel ms, launches)."""
+    import structured_rotations_b200 as H
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        plan.apply(x, y)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for a, b in ev:
+        a.record(stream)
+        plan.apply(x, y)
+        b.record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    elapsed = t0.elapsed_time(t1)
+    kern = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    return elapsed, kern, steps, H.last_kernel()
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import structured_rotations_b200 as H
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=device)
+        dist = tdist
+
+    w = W.get(args.workload)
+    rows, d = w.rows, w.d
+    plan = make_plan(args.workload, H, W)
+    t = time.time()
+    enc = W.draw_encoded(w, rank * rows, rows)       # this rank's shard of the global batch
+    log(f"rank {rank}: generated {rows}x{d} input in {time.time() - t:.1f}s")
+    x = to_device_bf16(enc, torch, device)
+    y = torch.empty_like(x)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    elapsed, kern_ms, launches, kname = time_apply(plan, x, y, args.steps, args.warmup, torch, dist)
+    clocks = sampler.stop()
+
+    if dist is not None:
+        tm = torch.tensor([elapsed], device=device, dtype=torch.float64)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        elapsed = float(tm.item())
+    step_ms = elapsed / args.steps
+    value = world * rows * args.steps / (elapsed / 1e3)
+    bytes_per_launch = 2 * rows * d * 2
+    peak, peak_kind = peaks()
+    achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9
+    traffic = recorded_traffic(kname, args.workload)
+
+    # end to end through the public API: pinned host rows in, pinned host rows out
+    xh = torch.from_numpy(enc.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        x.copy_(xh, non_blocking=True); plan.apply(x, y); yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        x.copy_(xh, non_blocking=True)
+        plan.apply(x, y)
+        yh.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        tm = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+    e2e = {"value": world * rows * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
+           "path": "pinned host -> device copy, harp_apply, device -> pinned host copy, one stream"}
+    del xh, yh
+
+    also = []
+    if not args.no_extra and rank == 0 and world == 1:
+        for name in ("c3_64k", "c5"):
+            ww = W.get(name)
+            p2 = make_plan(name, H, W)
+            e2 = W.draw_encoded(ww, 0, ww.rows)
+            x2 = to_device_bf16(e2, torch, device)
+            y2 = torch.empty_like(x2)
+            st = max(3, args.steps // 4)
+            el, km, _, kn = time_apply(p2, x2, y2, st, max(3, args.warmup // 2), torch)
+            b2 = 2 * ww.rows * ww.d * 2
+            also.append({"workload": WORKLOAD_TEXT[name], "rows_per_s": ww.rows * st / (el / 1e3),
+                         "hbm_gbs": b2 / (km / 1e3) / 1e9, "hbm_frac": b2 / (km / 1e3) / 1e9 / peak,
+                         "kernel": kn, "kernel_ms": km})
+            del x2, y2, p2
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        cpu = cpu_baseline(args, W)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "d": d, "schedule": list(w.schedule),
+                   "rows_per_gpu": rows, "io_dtype": "bf16", "parallelism": f"row shards x{world}",
+                   "l2": "inputs 512 MiB per step > 126 MB L2; no flush"},
+        "hbm_gbs": achieved, "hbm_frac": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth", "kernel": kname,
+                     "algorithmic_bytes_per_launch": bytes_per_launch, "kernel_ms": kern_ms},
+        "clocks": clocks, "gpu_launches": launches, "e2e": e2e,
+        "cpu_baseline": cpu, "also": also,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,203 @@
+/*
+ * harp.h — C ABI of libharp, a B200 (sm_100a) implementation of the HARP
+ * stride-staged block-orthogonal rotation.
+ *
+ * The operation (HARP technical summary, gist.science, "Technical Summary: HARP
+ * (Hadamard-Preconditioned Adaptive Rotation Processor)"):
+ *   §2.1 Core Architecture — a mixed-radix schedule b = (b_0, ..., b_{m-1}) with
+ *        prod b_t = d; stage t applies a block-diagonal orthogonal matrix to
+ *        groups of b_t coordinates separated by a stride permutation.
+ *   §2.2 Hadamard Preconditioning — each block is B_{t,c}(theta) = Q_{t,c}(theta)
+ *        G_{b_t}; G is the normalized Sylvester Hadamard for power-of-two radices
+ *        and a QR fallback of a fixed Gaussian matrix otherwise; Q is a Givens
+ *        rotation for b_t = 2 and a Cayley map for b_t > 2; theta = 0 recovers
+ *        the fixed randomized Hadamard transform.
+ *   §2.4 Deployment Efficiency — theta may be stored as int8.
+ *   Abstract — a two-sided processor: a rotation on each side of a weight matrix.
+ *
+ * Conventions fixed by this library (the pages leave them open):
+ *   strides      s_t = prod_{j<t} b_j; index i = sum_t i_t s_t, digit 0 least
+ *                significant; stage t mixes digit t.  The group of stage t that
+ *                holds block c = lo + s_t*hi (0 <= lo < s_t) is the b_t coordinates
+ *                lo + s_t*(k + b_t*hi), k = 0..b_t-1.
+ *   transform    T = M_{m-1} ... M_1 M_0 S, where S = diag(+-1) and
+ *                (M_t x)[lo + s_t(k + b_t hi)] = sum_l B_{t,c}[k][l] x[lo + s_t(l + b_t hi)].
+ *   signs        s_i = -1 if bit 63 of the i-th SplitMix64 output of sign_seed is
+ *                set, +1 otherwise (SplitMix64: state += 0x9E3779B97F4A7C15, then
+ *                the published 64-bit finalizer).
+ *   mixers       power of two: G[k][l] = (-1)^popcount(k&l) / sqrt(b).  Otherwise
+ *                one matrix per radix value: b*b standard normals, row-major, from
+ *                the SplitMix64 stream seeded with (qr_seed ? qr_seed :
+ *                0x4841525000000000) + b, two outputs per entry, U = (u >> 11) 2^-53,
+ *                g = sqrt(-2 ln(1 - U1)) cos(2 pi U2); G = Q diag(sign(R_kk)) from the
+ *                Householder QR M = QR (sign(0) = +1).
+ *   theta layout stages t = 0..m-1 in order; within a stage, blocks c = 0..d/b_t-1;
+ *                per block p_t parameters: p_t = 1 (Givens angle) if b_t = 2, else
+ *                b_t(b_t-1)/2 entries of the strict upper triangle of A in
+ *                row-major order ((0,1), (0,2), ..., (0,b-1), (1,2), ...), with
+ *                A[j][i] = -A[i][j] and Q = (I - A)^{-1} (I + A).
+ *                Givens: Q = [[cos, -sin], [sin, cos]].
+ *   int8 theta   theta = q * scales[t] for every parameter of stage t.
+ *
+ * Memory and streams:
+ *   * Every pointer named "host" is host memory; every activation/weight/output
+ *     pointer is device memory owned by the caller.  The plan owns copies of theta,
+ *     the signs, the mixers and the materialized blocks.
+ *   * All device work is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Argument errors are returned synchronously and leave
+ *     the stream untouched.  Launch errors return HARP_ERR_CUDA; faults of earlier
+ *     work surface at the next synchronizing call.
+ *   * Rows are dense vectors of length d; row r starts at x + r*ld elements.
+ *     ld >= d.  bf16 rows must start on 16-byte boundaries for the vectorized paths
+ *     (the library falls back to a scalar kernel otherwise, never to the CPU).
+ */
+#ifndef HARP_H_
+#define HARP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HARP_API __attribute__((visibility("default")))
+#else
+#define HARP_API
+#endif
+
+#define HARP_MAX_STAGES 16
+#define HARP_MAX_RADIX 16
+#define HARP_MAX_DIM 32768
+
+typedef struct harp_plan_s* harp_plan_t;
+
+typedef enum {
+    HARP_OK = 0,
+    HARP_ERR_INVALID_ARG = 1,     /* null pointer, bad size, bad stride, partial aliasing */
+    HARP_ERR_SCHEDULE = 2,        /* prod b_t != d, radix outside [2, 16], too many stages */
+    HARP_ERR_UNSUPPORTED = 3,     /* dtype / direction value not known */
+    HARP_ERR_NOT_MATERIALIZED = 4,/* harp_apply before harp_materialize_blocks */
+    HARP_ERR_ALLOC = 5,           /* device or host allocation failed */
+    HARP_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
+    HARP_ERR_TIMEOUT = 7,         /* a bounded device-side wait gave up */
+    HARP_ERR_WRONG_DEVICE = 8     /* plan materialized on another device */
+} harp_status;
+
+typedef enum { HARP_THETA_F32 = 0, HARP_THETA_I8 = 1 } harp_theta_kind;
+typedef enum { HARP_F32 = 0, HARP_BF16 = 1 } harp_dtype;
+/* FORWARD: y = T x.  INVERSE: y = T^T x (exact inverse; T is orthogonal). */
+typedef enum { HARP_FORWARD = 0, HARP_INVERSE = 1 } harp_dir;
+
+/*
+ * harp_plan_create — validate a schedule and build the host side of a plan
+ * (§2.1 schedule, §2.2 blocks).  Host only: no CUDA call is made.
+ *   out        receives the new plan (unchanged on error).
+ *   d          dimension, 2 <= d <= HARP_MAX_DIM.
+ *   radices    host array of m radices, each in [2, HARP_MAX_RADIX], product d.
+ *   m          number of stages, 1 <= m <= HARP_MAX_STAGES.
+ *   kind       HARP_THETA_F32: theta is a host float array; HARP_THETA_I8: theta
+ *              is a host int8 array of codes and `scales` holds m floats.
+ *   theta      harp_theta_count(radices, m) parameters in the layout above; NULL
+ *              means all zeros (the fixed randomized Hadamard transform).
+ *   scales     m per-stage scales for HARP_THETA_I8, ignored (may be NULL) for F32.
+ *   sign_seed  seed of the sign diagonal S.
+ *   qr_seed    0 selects the default seed base for the non-power-of-two mixers.
+ * Returns HARP_ERR_SCHEDULE / HARP_ERR_INVALID_ARG on bad input, HARP_ERR_ALLOC if
+ * host memory runs out.  The plan copies everything it needs.
+ */
+HARP_API harp_status harp_plan_create(harp_plan_t* out, int64_t d, const int32_t* radices, int32_t m,
+                             harp_theta_kind kind, const void* theta, const float* scales,
+                             uint64_t sign_seed, uint64_t qr_seed);
+
+/*
+ * harp_materialize_blocks — upload theta (as stored: float or int8 codes plus
+ * scales), signs and mixers to the current device and build every block
+ * B_{t,c} = Q_{t,c}(theta) G_{b_t} on the device (§2.2; int8 codes are
+ * dequantized inside the kernel, §2.4).  Blocks are computed in double and stored
+ * as float32; the sign diagonal is folded into the stage-0 blocks.  Allocates
+ * device memory owned by the plan on first use.  Idempotent; a second call on
+ * another device returns HARP_ERR_WRONG_DEVICE.
+ */
+HARP_API harp_status harp_materialize_blocks(harp_plan_t plan, void* stream);
+
+/*
+ * harp_apply — y_r = T x_r (FORWARD) or y_r = T^T x_r (INVERSE) for rows r < rows
+ * (§2.1 stages, §2.2 blocks; the inverse is the exact change of basis back).
+ *   x, y        device pointers, element type `dtype` (HARP_F32: float,
+ *               HARP_BF16: bfloat16 bits); y may equal x (in place); any other
+ *               overlap of the two row ranges returns HARP_ERR_INVALID_ARG.
+ *   rows        number of rows; 0 is a no-op returning HARP_OK.
+ *   ld_x, ld_y  leading dimensions in elements, >= d.
+ * Arithmetic: inputs widened to fp32, every stage accumulated in fp32 with fused
+ * multiply-adds, the output rounded to `dtype` to nearest even.
+ */
+HARP_API harp_status harp_apply(harp_plan_t plan, const void* x, void* y, int64_t rows,
+                       int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
+                       void* stream);
+
+/*
+ * harp_two_sided_workspace_bytes — device workspace that harp_apply_two_sided
+ * needs for an n_out x n_in weight (two fp32 copies of it, 256-byte aligned).
+ */
+HARP_API size_t harp_two_sided_workspace_bytes(int64_t n_out, int64_t n_in);
+
+/*
+ * harp_apply_two_sided — W_out = T_U^T W T_V (HARP abstract: a two-sided
+ * processor; U acts on the output side, V on the input side of W).
+ *   planU       plan with d = n_out (rotation of the columns of W).
+ *   planV       plan with d = n_in (rotation of the rows of W).
+ *   W, W_out    device pointers, n_out rows of n_in elements, leading dimension
+ *               ld >= n_in, element type `dtype`.  W_out may equal W.
+ *   workspace   device memory of at least harp_two_sided_workspace_bytes(),
+ *               256-byte aligned; intermediates are kept in fp32 there.
+ * Rows of W take T_V^T, columns take T_U^T; the result is rounded once, at the end.
+ * The original weight is W = T_U W_out T_V^T.
+ */
+HARP_API harp_status harp_apply_two_sided(harp_plan_t planU, harp_plan_t planV, const void* W,
+                                 void* W_out, int64_t n_out, int64_t n_in, int64_t ld,
+                                 harp_dtype dtype, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/* harp_plan_destroy — free the plan and its device memory (synchronizes the
+ * device that owns it).  NULL is accepted. */
+HARP_API harp_status harp_plan_destroy(harp_plan_t plan);
+
+/* harp_status_string — static, human-readable name of a status code. */
+HARP_API const char* harp_status_string(harp_status s);
+
+/* harp_last_kernel — name of the last kernel this host thread launched through
+ * harp_apply / harp_apply_two_sided (static per-thread buffer). */
+HARP_API const char* harp_last_kernel(void);
+
+/* harp_last_error — detail of the last failing call on this host thread (static
+ * per-thread buffer, valid until the next call). */
+HARP_API const char* harp_last_error(void);
+
+/* ------------------------------------------------------------------------- */
+/* Host-side introspection: no device work, usable without a GPU.            */
+/* ------------------------------------------------------------------------- */
+
+/* Number of parameters of a schedule: sum_t (d/b_t) p_t; -1 if the schedule is
+ * invalid. */
+HARP_API int64_t harp_theta_count(const int32_t* radices, int32_t m);
+
+/* The first n outputs of SplitMix64 started at `seed` (host array out[n]). */
+HARP_API harp_status harp_splitmix64(uint64_t seed, int64_t n, uint64_t* out);
+
+/* The plan's base mixer G_radix in double, row-major, into host out[radix*radix];
+ * HARP_ERR_INVALID_ARG if no stage of the plan uses that radix. */
+HARP_API harp_status harp_plan_base_mixer(harp_plan_t plan, int32_t radix, double* out);
+
+/* The plan's sign diagonal as +1/-1 into host out[d]. */
+HARP_API harp_status harp_plan_signs(harp_plan_t plan, int8_t* out);
+
+/* Dimension, stage count and radices of a plan (radices: host out[HARP_MAX_STAGES]). */
+HARP_API harp_status harp_plan_shape(harp_plan_t plan, int64_t* d, int32_t* m, int32_t* radices);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HARP_H_ */

@@ -1,0 +1,125 @@
+// C entry points that run device work: argument checks and dispatch between the
+// specialized and the general row kernels, and the two-sided weight rotation
+// (HARP abstract: a two-sided orthogonal processor; W_out = T_U^T W T_V).
+#include <cstdlib>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "harp_internal.h"
+
+namespace {
+
+size_t esize(harp_dtype t) { return t == HARP_F32 ? 4 : 2; }
+
+harp_status check_device(const harp_plan_s* p) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return harp_fail(HARP_ERR_CUDA, "no CUDA device");
+    }
+    if (dev != p->device)
+        return harp_fail(HARP_ERR_WRONG_DEVICE, "plan materialized on device " + std::to_string(p->device) +
+                                                    ", current device is " + std::to_string(dev));
+    return HARP_OK;
+}
+
+// 0 = auto, 1 = simple only, 2 = fast only (fail if the shape has no fast kernel)
+int kernel_choice() {
+    const char* v = std::getenv("HARP_KERNEL");
+    if (!v) return 0;
+    if (!std::strcmp(v, "simple")) return 1;
+    if (!std::strcmp(v, "fast")) return 2;
+    return 0;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const char* pa = (const char*)a;
+    const char* pb = (const char*)b;
+    return pa < pb + nb && pb < pa + na;
+}
+
+}  // namespace
+
+extern "C" harp_status harp_apply(harp_plan_t p, const void* x, void* y, int64_t rows,
+                                  int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
+                                  void* stream) {
+    harp_clear_error();
+    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    if (dtype != HARP_F32 && dtype != HARP_BF16) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown dtype");
+    if (dir != HARP_FORWARD && dir != HARP_INVERSE) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown direction");
+    if (rows < 0) return harp_fail(HARP_ERR_INVALID_ARG, "rows < 0");
+    const int64_t d = p->desc.d;
+    if (ld_x < d || ld_y < d) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than d");
+    if (rows == 0) return HARP_OK;
+    if (!x || !y) return harp_fail(HARP_ERR_INVALID_ARG, "x or y is NULL");
+    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    harp_status st = check_device(p);
+    if (st != HARP_OK) return st;
+    const size_t es = esize(dtype);
+    if (x == y) {
+        if (ld_x != ld_y) return harp_fail(HARP_ERR_INVALID_ARG, "in-place apply needs ld_x == ld_y");
+    } else if (ranges_overlap(x, ((rows - 1) * ld_x + d) * es, y, ((rows - 1) * ld_y + d) * es)) {
+        return harp_fail(HARP_ERR_INVALID_ARG, "x and y overlap without being equal");
+    }
+    const int choice = kernel_choice();
+    if (choice != 1) {
+        st = launch_apply_fast(p, x, y, rows, ld_x, ld_y, dtype, dir, stream, dtype);
+        if (st != HARP_ERR_UNSUPPORTED || choice == 2) return st;
+        harp_clear_error();
+    }
+    return launch_apply_simple(p, x, y, rows, ld_x, ld_y, dtype, dtype, dir, stream);
+}
+
+extern "C" size_t harp_two_sided_workspace_bytes(int64_t n_out, int64_t n_in) {
+    if (n_out <= 0 || n_in <= 0) return 0;
+    const size_t one = ((size_t)n_out * (size_t)n_in * sizeof(float) + 255) & ~(size_t)255;
+    return 2 * one;
+}
+
+extern "C" harp_status harp_apply_two_sided(harp_plan_t pu, harp_plan_t pv, const void* W,
+                                            void* W_out, int64_t n_out, int64_t n_in, int64_t ld,
+                                            harp_dtype dtype, void* workspace, size_t ws_bytes,
+                                            void* stream) {
+    harp_clear_error();
+    if (!pu || !pv) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    if (dtype != HARP_F32 && dtype != HARP_BF16) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown dtype");
+    if (n_out <= 0 || n_in <= 0) return harp_fail(HARP_ERR_INVALID_ARG, "empty weight");
+    if (pu->desc.d != n_out) return harp_fail(HARP_ERR_INVALID_ARG, "planU dimension differs from n_out");
+    if (pv->desc.d != n_in) return harp_fail(HARP_ERR_INVALID_ARG, "planV dimension differs from n_in");
+    if (ld < n_in) return harp_fail(HARP_ERR_INVALID_ARG, "ld smaller than n_in");
+    if (!W || !W_out || !workspace) return harp_fail(HARP_ERR_INVALID_ARG, "NULL pointer");
+    if (((uintptr_t)workspace & 255) != 0) return harp_fail(HARP_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    if (ws_bytes < harp_two_sided_workspace_bytes(n_out, n_in))
+        return harp_fail(HARP_ERR_INVALID_ARG, "workspace too small");
+    if (!pu->materialized || !pv->materialized)
+        return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks on both plans");
+    harp_status st;
+    if ((st = check_device(pu)) != HARP_OK || (st = check_device(pv)) != HARP_OK) return st;
+    const size_t es = esize(dtype);
+    const size_t wbytes = ((n_out - 1) * ld + n_in) * es;
+    if (W != W_out && ranges_overlap(W, wbytes, W_out, wbytes))
+        return harp_fail(HARP_ERR_INVALID_ARG, "W and W_out overlap without being equal");
+    if (ranges_overlap(W, wbytes, workspace, ws_bytes) || ranges_overlap(W_out, wbytes, workspace, ws_bytes))
+        return harp_fail(HARP_ERR_INVALID_ARG, "workspace overlaps the weight");
+
+    float* ws1 = (float*)workspace;
+    float* ws2 = (float*)((char*)workspace + harp_two_sided_workspace_bytes(n_out, n_in) / 2);
+    // rows of W: w_r <- T_V^T w_r (fp32 out)
+    st = launch_apply_fast(pv, W, ws1, n_out, ld, n_in, dtype, HARP_INVERSE, stream, HARP_F32);
+    if (st == HARP_ERR_UNSUPPORTED) {
+        harp_clear_error();
+        st = launch_apply_simple(pv, W, ws1, n_out, ld, n_in, dtype, HARP_F32, HARP_INVERSE, stream);
+    }
+    if (st != HARP_OK) return st;
+    if ((st = launch_transpose(ws1, ws2, n_out, n_in, n_in, n_out, HARP_F32, HARP_F32, stream)) != HARP_OK)
+        return st;
+    // columns of W (rows of W^T): col <- T_U^T col
+    st = launch_apply_fast(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_INVERSE, stream, HARP_F32);
+    if (st == HARP_ERR_UNSUPPORTED) {
+        harp_clear_error();
+        st = launch_apply_simple(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_F32, HARP_INVERSE, stream);
+    }
+    if (st != HARP_OK) return st;
+    return launch_transpose(ws2, W_out, n_in, n_out, n_out, ld, HARP_F32, dtype, stream);
+}

@@ -1,0 +1,73 @@
+// Internal declarations shared by the host plan code and the CUDA launchers.
+#pragma once
+
+#include <cstdint>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "harp.h"
+
+struct StageDesc {
+    int32_t b;          // radix b_t
+    int32_t p;          // parameters per block (1 for b=2, b(b-1)/2 otherwise)
+    int64_t s;          // stride s_t = prod_{j<t} b_j
+    int64_t nblocks;    // d / b_t
+    int64_t theta_off;  // first parameter of the stage
+    int64_t block_off;  // first float of the stage's blocks (nblocks * b * b floats)
+    int32_t mixer_off;  // first double of G_{b_t} in the packed mixer table
+};
+
+struct PlanDesc {       // passed by value to kernels
+    int64_t d;
+    int32_t m;
+    StageDesc st[HARP_MAX_STAGES];
+};
+
+struct harp_plan_s {
+    PlanDesc desc;
+    harp_theta_kind kind;
+    std::vector<float> theta_f32;
+    std::vector<int8_t> theta_i8;
+    std::vector<float> scales;
+    uint64_t sign_seed = 0, qr_seed = 0;
+    std::vector<int8_t> signs;                  // +1 / -1, length d
+    std::vector<double> mixers;                 // packed G_b, row-major
+    std::map<int, int> mixer_index;             // radix -> offset into mixers
+    int64_t theta_total = 0;
+    int64_t block_floats = 0;
+
+    // device side (owned)
+    int device = -1;
+    bool materialized = false;
+    float* d_blocks = nullptr;        // signed blocks, [stage][c][k][l]
+    void* d_theta = nullptr;          // float or int8 codes, as stored
+    float* d_scales = nullptr;
+    double* d_mixers = nullptr;
+    int8_t* d_signs = nullptr;
+    int* d_status = nullptr;          // device error word (bounded waits)
+    void* fast = nullptr;             // fast-path state (see apply_fast.cu)
+};
+
+// error reporting (plan.cpp)
+harp_status harp_fail(harp_status s, const std::string& msg);
+void harp_clear_error();
+void harp_set_last_kernel(const char* name);
+
+// device helpers (materialize.cu)
+harp_status harp_device_free(harp_plan_s* p);
+
+// launchers (apply_simple.cu / transpose.cu)
+harp_status launch_apply_simple(const harp_plan_s* p, const void* x, void* y, int64_t rows,
+                                int64_t ld_x, int64_t ld_y, harp_dtype in_dtype,
+                                harp_dtype out_dtype, harp_dir dir, void* stream);
+harp_status launch_transpose(const void* src, void* dst, int64_t rows, int64_t cols,
+                             int64_t ld_src, int64_t ld_dst, harp_dtype in_dtype,
+                             harp_dtype out_dtype, void* stream);
+
+// fast path (apply_fast.cu): returns HARP_ERR_UNSUPPORTED when the shape has no
+// specialized kernel, in which case the caller uses the simple kernel.
+harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t rows,
+                              int64_t ld_x, int64_t ld_y, harp_dtype in_dtype, harp_dir dir,
+                              void* stream, harp_dtype out_dtype);
+void fast_state_free(harp_plan_s* p);

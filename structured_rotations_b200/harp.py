@@ -1,0 +1,247 @@
+"""ctypes binding of libharp (include/harp.h): argument marshalling only.
+
+Every step of the transform runs in the library's CUDA kernels; this module
+passes device pointers and the current CUDA stream through.  Loading fails
+loudly when libharp.so has not been built — there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("HARP_LIB", os.path.join(_HERE, "libharp.so"))
+
+HARP_OK = 0
+HARP_ERR_INVALID_ARG = 1
+HARP_ERR_SCHEDULE = 2
+HARP_ERR_UNSUPPORTED = 3
+HARP_ERR_NOT_MATERIALIZED = 4
+HARP_ERR_ALLOC = 5
+HARP_ERR_CUDA = 6
+HARP_ERR_TIMEOUT = 7
+HARP_ERR_WRONG_DEVICE = 8
+
+HARP_THETA_F32 = 0
+HARP_THETA_I8 = 1
+HARP_F32 = 0
+HARP_BF16 = 1
+HARP_FORWARD = 0
+HARP_INVERSE = 1
+
+MAX_STAGES = 16
+
+_c_i64 = ctypes.c_int64
+_c_i32 = ctypes.c_int32
+_c_u64 = ctypes.c_uint64
+_vp = ctypes.c_void_p
+
+
+class HarpError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {detail or status}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libharp handle (raises if the library is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libharp.so not found at {LIB_PATH}; build it with "
+                          f"`python -m structured_rotations_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "harp_plan_create": (_c_i32, [ctypes.POINTER(_vp), _c_i64, ctypes.POINTER(_c_i32), _c_i32,
+                                      _c_i32, _vp, ctypes.POINTER(ctypes.c_float), _c_u64, _c_u64]),
+        "harp_materialize_blocks": (_c_i32, [_vp, _vp]),
+        "harp_apply": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32, _vp]),
+        "harp_two_sided_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64]),
+        "harp_apply_two_sided": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp,
+                                          ctypes.c_size_t, _vp]),
+        "harp_plan_destroy": (_c_i32, [_vp]),
+        "harp_status_string": (ctypes.c_char_p, [_c_i32]),
+        "harp_last_error": (ctypes.c_char_p, []),
+        "harp_last_kernel": (ctypes.c_char_p, []),
+        "harp_theta_count": (_c_i64, [ctypes.POINTER(_c_i32), _c_i32]),
+        "harp_splitmix64": (_c_i32, [_c_u64, _c_i64, ctypes.POINTER(_c_u64)]),
+        "harp_plan_base_mixer": (_c_i32, [_vp, _c_i32, ctypes.POINTER(ctypes.c_double)]),
+        "harp_plan_signs": (_c_i32, [_vp, ctypes.POINTER(ctypes.c_int8)]),
+        "harp_plan_shape": (_c_i32, [_vp, ctypes.POINTER(_c_i64), ctypes.POINTER(_c_i32),
+                                     ctypes.POINTER(_c_i32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status: int, where: str):
+    if status != HARP_OK:
+        L = lib()
+        detail = (L.harp_last_error() or b"").decode()
+        name = L.harp_status_string(status).decode()
+        raise HarpError(status, where, detail or name)
+
+
+def _radices(schedule: Sequence[int]):
+    arr = (_c_i32 * len(schedule))(*[int(b) for b in schedule])
+    return arr
+
+
+def theta_count(schedule: Sequence[int]) -> int:
+    return int(lib().harp_theta_count(_radices(schedule), len(schedule)))
+
+
+def splitmix64(seed: int, n: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint64)
+    _check(lib().harp_splitmix64(_c_u64(seed), n, out.ctypes.data_as(ctypes.POINTER(_c_u64))),
+           "harp_splitmix64")
+    return out
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+_DTYPE = {"float32": HARP_F32, "bfloat16": HARP_BF16}
+
+
+def _dtype_code(t) -> int:
+    name = str(t.dtype).replace("torch.", "")
+    if name not in _DTYPE:
+        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    return _DTYPE[name]
+
+
+def _ld(t) -> int:
+    if t.dim() != 2:
+        raise ValueError("expected a 2-D tensor of rows")
+    if t.stride(1) != 1:
+        raise ValueError("rows must be contiguous (stride(1) == 1)")
+    return t.stride(0) if t.shape[0] > 1 else max(t.stride(0), t.shape[1])
+
+
+class Plan:
+    """One HARP rotation: schedule, parameters, signs, mixers and device blocks."""
+
+    def __init__(self, d: int, schedule: Sequence[int], theta=None, sign_seed: int = 0,
+                 qr_seed: int = 0, codes=None, scales=None):
+        L = lib()
+        self.d = int(d)
+        self.schedule = tuple(int(b) for b in schedule)
+        handle = _vp()
+        if codes is not None:
+            codes = np.ascontiguousarray(codes, dtype=np.int8)
+            scales = np.ascontiguousarray(scales, dtype=np.float32)
+            kind, ptr = HARP_THETA_I8, codes.ctypes.data
+            sptr = scales.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+            self._keep = (codes, scales)
+        else:
+            kind = HARP_THETA_F32
+            if theta is not None:
+                theta = np.ascontiguousarray(theta, dtype=np.float32)
+                ptr = theta.ctypes.data
+            else:
+                ptr = None
+            sptr = None
+            self._keep = (theta,)
+        st = L.harp_plan_create(ctypes.byref(handle), self.d, _radices(self.schedule),
+                                len(self.schedule), kind, ptr, sptr, _c_u64(sign_seed), _c_u64(qr_seed))
+        _check(st, "harp_plan_create")
+        self._h = handle
+
+    @property
+    def handle(self):
+        return self._h
+
+    def materialize(self, stream=None) -> "Plan":
+        _check(lib().harp_materialize_blocks(self._h, _stream_handle(stream)), "harp_materialize_blocks")
+        return self
+
+    def apply(self, x, y=None, direction: str = "forward", stream=None, rows: Optional[int] = None):
+        """y = T x (forward) or T^T x (inverse) row by row; y defaults to a new tensor."""
+        import torch
+        if y is None:
+            y = torch.empty_like(x)
+        if x.dtype != y.dtype:
+            raise TypeError("x and y must share a dtype")
+        if x.shape[-1] != self.d or y.shape[-1] != self.d:
+            raise ValueError(f"last dimension must be d={self.d}")
+        n = x.shape[0] if rows is None else rows
+        d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
+        _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
+                                _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
+        return y
+
+    def base_mixer(self, radix: int) -> np.ndarray:
+        out = np.empty((radix, radix), dtype=np.float64)
+        _check(lib().harp_plan_base_mixer(self._h, radix, out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))),
+               "harp_plan_base_mixer")
+        return out
+
+    def signs(self) -> np.ndarray:
+        out = np.empty(self.d, dtype=np.int8)
+        _check(lib().harp_plan_signs(self._h, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int8))),
+               "harp_plan_signs")
+        return out
+
+    def shape(self):
+        d = _c_i64()
+        m = _c_i32()
+        r = (_c_i32 * MAX_STAGES)()
+        _check(lib().harp_plan_shape(self._h, ctypes.byref(d), ctypes.byref(m), r), "harp_plan_shape")
+        return d.value, tuple(r[: m.value])
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().harp_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def last_kernel() -> str:
+    """Name of the last kernel launched by this thread through the library."""
+    return (lib().harp_last_kernel() or b"").decode()
+
+
+def workspace_bytes(n_out: int, n_in: int) -> int:
+    return int(lib().harp_two_sided_workspace_bytes(n_out, n_in))
+
+
+def apply_two_sided(plan_u: Plan, plan_v: Plan, w, w_out=None, workspace=None, stream=None):
+    """W_out = T_U^T W T_V (U on the output side, V on the input side)."""
+    import torch
+    n_out, n_in = w.shape
+    if w_out is None:
+        w_out = torch.empty_like(w)
+    need = workspace_bytes(n_out, n_in)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=w.device)
+    ld = _ld(w)
+    if _ld(w_out) != ld:
+        raise ValueError("W and W_out must share a leading dimension")
+    _check(lib().harp_apply_two_sided(plan_u.handle, plan_v.handle, w.data_ptr(), w_out.data_ptr(),
+                                      n_out, n_in, ld, _dtype_code(w), workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream_handle(stream)), "harp_apply_two_sided")
+    return w_out

@@ -1,0 +1,125 @@
+"""CPU tests of libharp's host side through the C ABI: the library loads, exports
+every entry point that include/harp.h declares, and its host logic (schedule
+validation, SplitMix64, signs, base mixers, theta counts) agrees with the oracle,
+which was written separately.  No compute call is made without a GPU."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import harp_oracle as O
+import structured_rotations_b200 as H
+from structured_rotations_b200 import harp as HB
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        src = open(os.path.join(ROOT, "include", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names.update(re.findall(r"\b(harp_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = H.lib()
+    names = _declared_functions()
+    assert len(names) >= 13
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    L = H.lib()
+    for code, name in [(0, b"HARP_OK"), (2, b"HARP_ERR_SCHEDULE"), (4, b"HARP_ERR_NOT_MATERIALIZED"),
+                       (7, b"HARP_ERR_TIMEOUT")]:
+        assert L.harp_status_string(code) == name
+
+
+def test_splitmix64_matches_published_and_oracle():
+    got = H.splitmix64(0, 4).tolist()
+    assert got == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F, 0xF88BB8A8724C81EC]
+    assert H.splitmix64(3003, 64).tolist() == O.splitmix64(3003, 64)
+
+
+@pytest.mark.parametrize("schedule", [(8, 8), (2,) * 6, (8, 8, 8, 8), (8, 8, 8, 5, 2),
+                                      (8, 8, 8, 8, 2), (8, 8, 8, 8, 7), (16, 3, 11)])
+def test_theta_count_matches_oracle(schedule):
+    assert H.theta_count(schedule) == O.theta_count(schedule)
+
+
+@pytest.mark.parametrize("b", [2, 3, 4, 5, 7, 8, 11, 16])
+def test_base_mixers_match_oracle(b):
+    plan = H.Plan(b * 2, (b, 2), sign_seed=1)
+    np.testing.assert_allclose(plan.base_mixer(b), O.base_mixer(b), atol=1e-14, rtol=0)
+
+
+def test_qr_seed_is_honoured():
+    plan = H.Plan(10, (5, 2), qr_seed=99)
+    np.testing.assert_allclose(plan.base_mixer(5), O.qr_mixer(5, 99), atol=1e-14, rtol=0)
+
+
+@pytest.mark.parametrize("d,schedule,seed", [(4096, (8, 8, 8, 8), 3002), (28672, (8, 8, 8, 8, 7), 1),
+                                             (64, (2,) * 6, 3001)])
+def test_signs_match_oracle(d, schedule, seed):
+    plan = H.Plan(d, schedule, sign_seed=seed)
+    np.testing.assert_array_equal(plan.signs().astype(float), O.sign_vector(d, seed))
+    assert plan.shape() == (d, schedule)
+
+
+@pytest.mark.parametrize("d,schedule,code", [
+    (64, (8, 4), HB.HARP_ERR_SCHEDULE),            # product differs from d
+    (64, (64,), HB.HARP_ERR_SCHEDULE),             # radix above 16
+    (2, (1, 2), HB.HARP_ERR_SCHEDULE),             # radix below 2
+    (65536, (16, 16, 16, 16), HB.HARP_ERR_INVALID_ARG),  # d above the maximum
+    (1, (1,), HB.HARP_ERR_INVALID_ARG),
+])
+def test_plan_validation_errors(d, schedule, code):
+    with pytest.raises(HB.HarpError) as e:
+        H.Plan(d, schedule)
+    assert e.value.status == code
+
+
+def test_too_many_stages():
+    with pytest.raises(HB.HarpError) as e:
+        H.Plan(2 ** 17, (2,) * 17)
+    assert e.value.status in (HB.HARP_ERR_SCHEDULE, HB.HARP_ERR_INVALID_ARG)
+
+
+def test_int8_without_scales_rejected():
+    L = H.lib()
+    h = ctypes.c_void_p()
+    codes = np.zeros(O.theta_count((8, 8)), dtype=np.int8)
+    st = L.harp_plan_create(ctypes.byref(h), 64, HB._radices((8, 8)), 2, HB.HARP_THETA_I8,
+                            codes.ctypes.data, None, 0, 0)
+    assert st == HB.HARP_ERR_INVALID_ARG
+
+
+def test_apply_before_materialize_is_reported_without_touching_a_device():
+    L = H.lib()
+    plan = H.Plan(64, (8, 8))
+    st = L.harp_apply(plan.handle, ctypes.c_void_p(16), ctypes.c_void_p(16), 4, 64, 64,
+                      HB.HARP_F32, HB.HARP_FORWARD, None)
+    assert st == HB.HARP_ERR_NOT_MATERIALIZED
+    assert b"materialize" in L.harp_last_error()
+    # argument errors come first and never reach the device
+    assert L.harp_apply(plan.handle, None, None, 0, 64, 64, 0, 0, None) == HB.HARP_OK
+    assert L.harp_apply(plan.handle, None, None, 4, 63, 64, 0, 0, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_apply(plan.handle, None, None, 4, 64, 64, 7, 0, None) == HB.HARP_ERR_UNSUPPORTED
+    assert L.harp_apply(plan.handle, None, None, 4, 64, 64, 0, 5, None) == HB.HARP_ERR_UNSUPPORTED
+    assert L.harp_apply(None, None, None, 4, 64, 64, 0, 0, None) == HB.HARP_ERR_INVALID_ARG
+
+
+def test_two_sided_workspace_bytes():
+    assert H.workspace_bytes(28672, 8192) == 2 * 28672 * 8192 * 4
+    assert H.workspace_bytes(3, 5) == 2 * 256
+    assert H.workspace_bytes(0, 5) == 0
+
+
+def test_destroy_null_is_ok():
+    assert H.lib().harp_plan_destroy(None) == HB.HARP_OK

@@ -26,8 +26,10 @@ Seeds: data = 1000 + k, theta = 2000 + k, sign seed = 3000 + k for workload k.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
 import math
+import os
 from typing import Optional, Sequence
 
 import numpy as np
@@ -117,16 +119,21 @@ def encode_bf16(x: np.ndarray) -> np.ndarray:
     magnitude is below bf16's smallest normal are handled by scaling, so the
     result is correctly rounded there too.
     """
-    x = np.ascontiguousarray(x, dtype=np.float64)
-    bits = x.view(np.uint64)
+    x = np.asarray(x, dtype=np.float64)
+    bits = np.array(x, dtype=np.float64, copy=True).view(np.uint64)
     # add half an ulp of the 7-bit mantissa (minus one) plus the lowest kept bit,
     # then clear the 45 dropped bits: round-to-nearest-even on the bit pattern
-    keep_lsb = (bits >> np.uint64(45)) & np.uint64(1)
-    r = bits + np.uint64((1 << 44) - 1) + keep_lsb
-    r &= ~np.uint64((1 << 45) - 1)
-    out = (r.view(np.float64).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
-    tiny = (np.abs(x) < 2.0 ** -126) & (x != 0)
-    if np.any(tiny):
+    lsb = bits >> np.uint64(45)
+    lsb &= np.uint64(1)
+    bits += lsb
+    del lsb
+    bits += np.uint64((1 << 44) - 1)
+    bits &= ~np.uint64((1 << 45) - 1)
+    f32 = bits.view(np.float64).astype(np.float32)
+    del bits
+    out = (f32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    if x.size and np.abs(x).min() < 2.0 ** -126:
+        tiny = (np.abs(x) < 2.0 ** -126) & (x != 0)
         t = np.rint(x[tiny] * 2.0 ** 133) * 2.0 ** -133
         out[tiny] = (t.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
     return out
@@ -167,6 +174,37 @@ def _draw_block(w: Workload, block: int, d: int) -> np.ndarray:
     return x
 
 
+def _rows_f64(w: Workload, row_start: int, row_count: int, d: int) -> np.ndarray:
+    out = np.empty((row_count, d), dtype=np.float64)
+    if row_count == 0:
+        return out
+    b0 = row_start // ROW_BLOCK
+    b1 = (row_start + row_count - 1) // ROW_BLOCK
+
+    def one(blk):
+        x = _draw_block(w, blk, d)
+        lo = max(row_start, blk * ROW_BLOCK) - blk * ROW_BLOCK
+        hi = min(row_start + row_count, (blk + 1) * ROW_BLOCK) - blk * ROW_BLOCK
+        pos = blk * ROW_BLOCK + lo - row_start
+        out[pos:pos + (hi - lo)] = x[lo:hi]
+
+    blocks = range(b0, b1 + 1)
+    if len(blocks) > 2:
+        with cf.ThreadPoolExecutor(max_workers=_threads()) as ex:
+            list(ex.map(one, blocks))
+    else:
+        for blk in blocks:
+            one(blk)
+    return out
+
+
+def _threads() -> int:
+    try:
+        return max(1, min(32, len(os.sched_getaffinity(0))))
+    except AttributeError:
+        return max(1, min(32, os.cpu_count() or 1))
+
+
 def draw_rows(w: Workload, row_start: int = 0, row_count: Optional[int] = None,
               d: Optional[int] = None) -> np.ndarray:
     """Rows [row_start, row_start+row_count) of workload ``w`` as float64 values
@@ -175,31 +213,46 @@ def draw_rows(w: Workload, row_start: int = 0, row_count: Optional[int] = None,
     d = w.d if d is None else d
     if row_count is None:
         row_count = w.rows - row_start
-    out = np.empty((row_count, d), dtype=np.float64)
-    if row_count == 0:
-        return out
-    b0 = row_start // ROW_BLOCK
-    b1 = (row_start + row_count - 1) // ROW_BLOCK
-    pos = 0
-    for blk in range(b0, b1 + 1):
-        x = _draw_block(w, blk, d)
-        lo = max(row_start, blk * ROW_BLOCK) - blk * ROW_BLOCK
-        hi = min(row_start + row_count, (blk + 1) * ROW_BLOCK) - blk * ROW_BLOCK
-        x = x[lo:hi]
-        out[pos:pos + (hi - lo)] = x
-        pos += hi - lo
+    enc = draw_encoded(w, row_start, row_count, d)
     if w.dtype == "bf16":
-        return decode_bf16(encode_bf16(out))
-    return out.astype(np.float32).astype(np.float64)
+        return decode_bf16(enc)
+    return enc.astype(np.float64)
 
 
 def draw_encoded(w: Workload, row_start: int = 0, row_count: Optional[int] = None,
                  d: Optional[int] = None) -> np.ndarray:
-    """Same rows as :func:`draw_rows`, in storage form (float32 or bf16 bits)."""
-    x = draw_rows(w, row_start, row_count, d)
-    if w.dtype == "bf16":
+    """Rows [row_start, row_start+row_count) in storage form: float32, or bf16 bit
+    patterns (uint16) rounded to nearest even from the float64 draws."""
+    d = w.d if d is None else d
+    if row_count is None:
+        row_count = w.rows - row_start
+    out = np.empty((row_count, d), dtype=np.uint16 if w.dtype == "bf16" else np.float32)
+    step = 16 * ROW_BLOCK
+    # draw and encode in slabs so float64 temporaries stay small
+    for a in range(0, row_count, step):
+        n = min(step, row_count - a)
+        x = _rows_f64(w, row_start + a, n, d)
+        if w.dtype == "bf16":
+            out[a:a + n] = _encode_threads(x)
+        else:
+            out[a:a + n] = x.astype(np.float32)
+    return out
+
+
+def _encode_threads(x: np.ndarray) -> np.ndarray:
+    n = x.shape[0]
+    if n < 512:
         return encode_bf16(x)
-    return x.astype(np.float32)
+    parts = np.array_split(np.arange(n), _threads())
+    out = np.empty(x.shape, dtype=np.uint16)
+
+    def one(idx):
+        if idx.size:
+            out[idx[0]:idx[-1] + 1] = encode_bf16(x[idx[0]:idx[-1] + 1])
+
+    with cf.ThreadPoolExecutor(max_workers=_threads()) as ex:
+        list(ex.map(one, parts))
+    return out
 
 
 def draw_weight(w: Workload) -> np.ndarray:
