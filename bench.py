@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--rows", type=int, default=0, help="rows per GPU (default: the workload's; "
+                    "smaller values are for profiling captures, not bench lines)")
     return ap.parse_args()
 
 
@@ -256,53 +258,8 @@ def time_apply(plan, x, y, steps, warmup, torch, dist=None):
     return elapsed, kern, steps, H.last_kernel()
 
 
-def run_ours(args):
+def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
     import numpy as np
-    import torch
-    import structured_rotations_b200 as H
-    import workloads as W
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        log(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as tdist
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                 device_id=device)
-        dist = tdist
-
-    w = W.get(args.workload)
-    rows, d = w.rows, w.d
-    plan = make_plan(args.workload, H, W)
-    t = time.time()
-    enc = W.draw_encoded(w, rank * rows, rows)       # this rank's shard of the global batch
-    log(f"rank {rank}: generated {rows}x{d} input in {time.time() - t:.1f}s")
-    x = to_device_bf16(enc, torch, device)
-    y = torch.empty_like(x)
-
-    sampler = ClockSampler(local)
-    sampler.start()
-    elapsed, kern_ms, launches, kname = time_apply(plan, x, y, args.steps, args.warmup, torch, dist)
-    clocks = sampler.stop()
-
-    if dist is not None:
-        tm = torch.tensor([elapsed], device=device, dtype=torch.float64)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        elapsed = float(tm.item())
-    step_ms = elapsed / args.steps
-    value = world * rows * args.steps / (elapsed / 1e3)
-    bytes_per_launch = 2 * rows * d * 2
-    peak, peak_kind = peaks()
-    achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9
-    traffic = recorded_traffic(kname, args.workload)
-
-    # end to end through the public API: pinned host rows in, pinned host rows out
     xh = torch.from_numpy(enc.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     stream = torch.cuda.current_stream()
@@ -328,6 +285,57 @@ def run_ours(args):
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "path": "pinned host -> device copy, harp_apply, device -> pinned host copy, one stream"}
     del xh, yh
+    return e2e
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import structured_rotations_b200 as H
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        log(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=device)
+        dist = tdist
+
+    w = W.get(args.workload, args.rows or None)
+    rows, d = w.rows, w.d
+    plan = make_plan(args.workload, H, W)
+    t = time.time()
+    enc = W.draw_encoded(w, rank * rows, rows)       # this rank's shard of the global batch
+    log(f"rank {rank}: generated {rows}x{d} input in {time.time() - t:.1f}s")
+    x = to_device_bf16(enc, torch, device)
+    y = torch.empty_like(x)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    elapsed, kern_ms, launches, kname = time_apply(plan, x, y, args.steps, args.warmup, torch, dist)
+    clocks = sampler.stop()
+
+    if dist is not None:
+        tm = torch.tensor([elapsed], device=device, dtype=torch.float64)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        elapsed = float(tm.item())
+    step_ms = elapsed / args.steps
+    value = world * rows * args.steps / (elapsed / 1e3)
+    bytes_per_launch = 2 * rows * d * 2
+    peak, peak_kind = peaks()
+    achieved = bytes_per_launch / (kern_ms / 1e3) / 1e9
+    traffic = recorded_traffic(kname, args.workload)
+
+    # end to end through the public API: pinned host rows in, pinned host rows out
+    e2e = end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows) if args.e2e_steps > 0 else None
 
     also = []
     if not args.no_extra and rank == 0 and world == 1:
