@@ -160,6 +160,35 @@ HARP_API harp_status harp_apply_two_sided(harp_plan_t planU, harp_plan_t planV, 
                                  harp_dtype dtype, void* workspace, size_t ws_bytes,
                                  void* stream);
 
+/*
+ * harp_apply_two_sided_noalloc — the same W_out = T_U^T W T_V as
+ * harp_apply_two_sided, for callers that cannot allocate device memory when they
+ * rotate a weight (code that runs inside a memory pool or arena it does not own,
+ * inside a capture region, or in a host runtime that exposes no allocator to
+ * plugins).  It needs no workspace argument: the two fp32 intermediates live in a
+ * fixed array of HARP_NOALLOC_SCRATCH_BYTES inside the library's device image,
+ * which every GPU that loads the library holds until the process exits.  The
+ * paper has no counterpart of this entry point; it exists for such callers only.
+ *   Limit: n_out * n_in <= HARP_NOALLOC_SCRATCH_BYTES / 8 elements (4,194,304),
+ *          else HARP_ERR_INVALID_ARG and nothing is launched.
+ *   First call on a device: looks up the array's device address
+ *          (cudaGetSymbolAddress) with that device current; make that first call
+ *          before any stream capture.
+ *   Sharing: all calls use the same array; calls whose work overlaps on the GPU
+ *          (different streams or host threads) race on it and must be serialized
+ *          by the caller.  No part of the array needs to start at zero.
+ *   It calls no cudaMalloc, cudaFree or other allocating routine.  Other arguments
+ *   and errors are those of harp_apply_two_sided.
+ */
+#define HARP_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+HARP_API harp_status harp_apply_two_sided_noalloc(harp_plan_t planU, harp_plan_t planV,
+                                                  const void* W, void* W_out, int64_t n_out,
+                                                  int64_t n_in, int64_t ld, harp_dtype dtype,
+                                                  void* stream);
+
+/* harp_noalloc_scratch_bytes — size of that static array (HARP_NOALLOC_SCRATCH_BYTES). */
+HARP_API size_t harp_noalloc_scratch_bytes(void);
+
 /* harp_plan_destroy — free the plan and its device memory (synchronizes the
  * device that owns it).  NULL is accepted. */
 HARP_API harp_status harp_plan_destroy(harp_plan_t plan);

@@ -66,6 +66,9 @@ def lib():
         "harp_two_sided_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64]),
         "harp_apply_two_sided": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp,
                                           ctypes.c_size_t, _vp]),
+        "harp_apply_two_sided_noalloc": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32,
+                                                  _vp]),
+        "harp_noalloc_scratch_bytes": (ctypes.c_size_t, []),
         "harp_plan_destroy": (_c_i32, [_vp]),
         "harp_status_string": (ctypes.c_char_p, [_c_i32]),
         "harp_last_error": (ctypes.c_char_p, []),
