@@ -189,6 +189,12 @@ HARP_API harp_status harp_apply_two_sided_noalloc(harp_plan_t planU, harp_plan_t
 /* harp_noalloc_scratch_bytes — size of that static array (HARP_NOALLOC_SCRATCH_BYTES). */
 HARP_API size_t harp_noalloc_scratch_bytes(void);
 
+/* harp_plan_device_status — synchronizes the plan's device and reports whether any
+ * bounded device-side wait of a kernel launched with this plan gave up since the
+ * last call: HARP_ERR_TIMEOUT if one did (the flag is then cleared), HARP_OK if
+ * not, HARP_ERR_NOT_MATERIALIZED before materialization. */
+HARP_API harp_status harp_plan_device_status(harp_plan_t plan);
+
 /* harp_plan_destroy — free the plan and its device memory (synchronizes the
  * device that owns it).  NULL is accepted. */
 HARP_API harp_status harp_plan_destroy(harp_plan_t plan);

@@ -174,3 +174,20 @@ extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream_) {
     p->materialized = true;
     return HARP_OK;
 }
+
+extern "C" harp_status harp_plan_device_status(harp_plan_t p) {
+    harp_clear_error();
+    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    if (!p->materialized || !p->d_status) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "plan not materialized");
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(p->device);
+    int flag = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&flag, p->d_status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && flag) e = cudaMemset(p->d_status, 0, sizeof(int));
+    cudaSetDevice(prev);
+    if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    if (flag) return harp_fail(HARP_ERR_TIMEOUT, "a bounded device wait gave up");
+    return HARP_OK;
+}

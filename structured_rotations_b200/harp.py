@@ -69,6 +69,7 @@ def lib():
         "harp_apply_two_sided_noalloc": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32,
                                                   _vp]),
         "harp_noalloc_scratch_bytes": (ctypes.c_size_t, []),
+        "harp_plan_device_status": (_c_i32, [_vp]),
         "harp_plan_destroy": (_c_i32, [_vp]),
         "harp_status_string": (ctypes.c_char_p, [_c_i32]),
         "harp_last_error": (ctypes.c_char_p, []),
@@ -190,6 +191,11 @@ class Plan:
         _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
                                 _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
         return y
+
+    def device_status(self) -> None:
+        """Synchronize and raise HarpError(HARP_ERR_TIMEOUT) if a bounded device
+        wait of a kernel launched with this plan gave up."""
+        _check(lib().harp_plan_device_status(self._h), "harp_plan_device_status")
 
     def base_mixer(self, radix: int) -> np.ndarray:
         out = np.empty((radix, radix), dtype=np.float64)

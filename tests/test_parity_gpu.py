@@ -290,3 +290,14 @@ def test_materialize_is_idempotent_and_blocks_are_reused():
     enc = full_input("c1", 1024)
     out = run(gp, enc, "forward")
     check(out, tr.forward(decode(enc)), decode(enc), "after second materialize")
+
+
+def test_bench_shape_uses_the_specialized_kernel_and_no_wait_gave_up():
+    gp, tr = plans("c2")
+    enc = W.draw_encoded(W.get("c2"), 0, 4096 + 5)
+    out = run(gp, enc, "forward")
+    assert H.last_kernel() == "harp_fast_d4096_fwd_kernel"
+    gp.device_status()
+    idx = W.sample_rows(enc.shape[0], 300)
+    x = decode(enc[idx])
+    check(out[idx], tr.forward(x), x, "fast kernel 4101 rows")
