@@ -24,9 +24,12 @@
 // Every shared-memory access pattern below is XOR-swizzled to be bank-conflict
 // free; the derivations are next to each index function.
 #include <cstdio>
+#include <mutex>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "harp_internal.h"
 
@@ -39,18 +42,20 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kEFloats = 2 * 16 * 32 * 32;   // exchange tile E[half][row][a_local][pos]
 constexpr int kSFloats = 16 * 32 * 32;       // send buffer S[row][a_local][pos], reused as bf16 output staging
 constexpr int kHalfBytes = kSFloats * 4;     // 65536
-constexpr size_t kSmemBytes = (size_t)(kEFloats + kSFloats) * 4 + 64;
+constexpr int kXBytes = 16 * 128;            // one 16-row x 64-column bf16 input box per warp
+constexpr int kXOffset = (kEFloats + kSFloats) * 4;          // 196608, 1024-aligned
+constexpr int kBarOffset = kXOffset + kWarps * kXBytes;      // 229376
+constexpr size_t kSmemBytes = (size_t)kBarOffset + 8 * (kWarps + 1) + 1024;   // + alignment slack
 constexpr long long kWaitLimit = 1ll << 26;  // mbarrier polls before giving up
 
 struct FastParams {
-    const uint32_t* x;       // bf16 rows viewed as 32-bit words (pairs)
     __nv_bfloat16* y;
-    int64_t rows, ldx_w, ldy;  // ldx in 32-bit words, ldy in elements
+    int64_t rows, ldy;       // ldy in elements
     int ntiles;
     const float2* pk0;       // stage-0 B fragments, [block][lane]
-    const float* blk1;       // stage-1 blocks, row-major [block][8][8]
+    const float4* pk1;       // stage-1 blocks, lane-interleaved (see pack_interleaved_kernel)
     const float2* pk2;       // stage-2 B fragments
-    const float* blk3;       // stage-3 blocks
+    const float4* pk3;       // stage-3 blocks, lane-interleaved
     int* status;
 };
 
@@ -138,10 +143,12 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* s
         : "memory");
 }
 
-__device__ __forceinline__ uint32_t ldg_nc_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
+// 2-D tiled TMA load of one box into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int col, int row, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(col), "r"(row), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ------------------------------------------------------ shared layouts ---
@@ -165,11 +172,22 @@ __device__ __forceinline__ int s_index(int row, int a_local, int beta) {
 }
 
 // Output staging O[row][a_local][beta'] (bf16) with beta' = 8 i2 + i3, stored in 16-byte
-// chunks indexed by i2 ^ ((row & 1) << 2): a quarter-warp stores rows g in {2k, 2k+1}
-// with i2 = q + 4s, which lands in 8 distinct chunks.
+// chunks indexed by i2 ^ h, h = 2 ((a_local >> 3) & 3) ^ 4 (row & 1).
+//  - phase B stores a 16-byte chunk per lane (a_local fixed, i2 = q + 4s, rows 2k and 2k+1
+//    in a quarter-warp): the row bit moves the chunk to the other half, 8 distinct chunks.
+//  - the store phase loads one word per thread with the row fixed, 8 consecutive beta'
+//    pairs and the 4 pencil quarters u = a_local >> 3: chunks (p >> 2) ^ 2u are 8 distinct
+//    values and p & 3 selects the word, 32 distinct banks.
 __device__ __forceinline__ int o_byte(int row, int a_local, int i2, int i3) {
-    const int chunk = i2 ^ ((row & 1) << 2);
+    const int chunk = i2 ^ ((((a_local >> 3) & 3) << 1) ^ ((row & 1) << 2));
     return ((row * 32 + a_local) * 64 + chunk * 8 + i3) * 2;
+}
+
+// Input staging: TMA writes a 16 x 128-byte box with the 128-byte swizzle, i.e. the
+// 16-byte chunk c of row r sits at chunk position c ^ (r & 7).  The lane that needs
+// elements 8j + 2q, 8j + 2q + 1 of row g reads word q of chunk j ^ g: 32 distinct banks.
+__device__ __forceinline__ int x_byte(int row, int j, int q) {
+    return row * 128 + ((j ^ (row & 7)) << 4) + 4 * q;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -180,45 +198,54 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ------------------------------------------------------------- kernel ---
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    harp_fast_d4096_fwd_kernel(FastParams p) {
-    extern __shared__ __align__(128) float smem[];
-    float* E = smem;
-    float* S = smem + kEFloats;
+    harp_fast_d4096_fwd_kernel(const __grid_constant__ CUtensorMap tmap_x, FastParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled TMA boxes
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    float* E = reinterpret_cast<float*>(base);
+    float* S = E + kEFloats;
     unsigned char* O = reinterpret_cast<unsigned char*>(S);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(S + kSFloats);
+    unsigned char* X = base + kXOffset;
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(base + kBarOffset);   // one per warp
+    uint64_t* bar = xbar + kWarps;                                      // exchange
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, q = lane & 3;
     const int r = (int)cluster_rank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    unsigned char* Xw = X + warp * kXBytes;
 
     if (tid == 0) mbar_init(bar, 1);
-    // the partner's view of our chunk half of its E, and the partner's barrier
+    if (lane == 0) mbar_init(xbar + warp, 1);
     const uint32_t remote_e = map_to_rank(smem_u32(E + r * kSFloats), (uint32_t)(r ^ 1));
     const uint32_t remote_bar = map_to_rank(smem_u32(bar), (uint32_t)(r ^ 1));
     cluster_arrive();
-    cluster_wait();     // barrier initialised on both CTAs
+    cluster_wait();     // barriers initialised on both CTAs
     cluster_arrive();   // "my E may be written": matched by the wait before the first send
 
-    uint32_t parity = 0;
+    // first input box of this warp: tile `pair`, task 0
+    if (lane == 0 && pair < p.ntiles) {
+        mbar_arrive_expect_tx(xbar + warp, kXBytes);
+        tma_load_2d(Xw, &tmap_x, 64 * (32 * r + 2 * warp), pair * kTile, xbar + warp);
+    }
+    uint32_t xparity = 0, parity = 0;
+
     for (int tile = pair; tile < p.ntiles; tile += npairs) {
         const int64_t row0 = (int64_t)tile * kTile;
         if (tid == 0) mbar_arrive_expect_tx(bar, kHalfBytes);
 
         // -------------------------------------------------- phase A ---
-        const int64_t rA = row0 + g, rB = row0 + g + 8;
-        const bool vA = rA < p.rows, vB = rB < p.rows;
 #pragma unroll 1
         for (int task = 0; task < 2; ++task) {
             const int beta = 32 * r + 2 * warp + task;
-            const uint32_t* xa = p.x + rA * p.ldx_w + 32 * beta + q;
-            const uint32_t* xb = p.x + rB * p.ldx_w + 32 * beta + q;
+            if (!mbar_wait(xbar + warp, xparity) && lane == 0) atomicExch(p.status, 1);
+            xparity ^= 1;
             uint32_t w0[8], w1[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {   // element 8j + 2q (+1) of the chunk
-                w0[j] = vA ? ldg_nc_u32(xa + 4 * j) : 0u;
-                w1[j] = vB ? ldg_nc_u32(xb + 4 * j) : 0u;
+            for (int j = 0; j < 8; ++j) {   // elements 8j + 2q, 8j + 2q + 1 of rows g, g + 8
+                w0[j] = *reinterpret_cast<const uint32_t*>(Xw + x_byte(g, j, q));
+                w1[j] = *reinterpret_cast<const uint32_t*>(Xw + x_byte(g + 8, j, q));
             }
             // stage 0 on tensor cores: group j = i1, slot q <-> i0 = 2q, slot q+4 <-> i0 = 2q+1;
             // output slot 2q <-> i0 = q, 2q+1 <-> i0 = q + 4.
@@ -236,14 +263,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) z[j][e] = d[e];
             }
+            // every lane has consumed its words: refill the box with the second chunk of this
+            // tile, or the first chunk of the next tile
+            __syncwarp();
+            if (lane == 0) {
+                const int ntile = task == 0 ? tile : tile + npairs;
+                if (ntile < p.ntiles) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(xbar + warp, kXBytes);
+                    tma_load_2d(Xw, &tmap_x, 64 * (32 * r + 2 * warp + (task ^ 1)), ntile * kTile, xbar + warp);
+                }
+            }
             // stage 1 in registers: this lane holds i1 = 0..7 of groups i0 = q + 4s for rows g, g+8
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
-                const float* blk = p.blk1 + (size_t)((q + 4 * s) + 8 * beta) * 64;
+                const float4* blk = p.pk1 + (size_t)((beta * 2 + s) * 8) * 8 + q;
 #pragma unroll
                 for (int o = 0; o < 8; ++o) {
-                    const float4 c0 = __ldg(reinterpret_cast<const float4*>(blk + o * 8));
-                    const float4 c1 = __ldg(reinterpret_cast<const float4*>(blk + o * 8 + 4));
+                    const float4 c0 = __ldg(blk + (o * 2 + 0) * 4);
+                    const float4 c1 = __ldg(blk + (o * 2 + 1) * 4);
                     const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                     float yA = 0.f, yB = 0.f;
 #pragma unroll
@@ -306,12 +344,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
                 const int i2 = q + 4 * s;
-                const float* blk = p.blk3 + (size_t)(a + 64 * i2) * 64;
+                const float4* blk = p.pk3 + (size_t)((a * 2 + s) * 8) * 8 + q;
                 float yA[8], yB[8];
 #pragma unroll
                 for (int o = 0; o < 8; ++o) {
-                    const float4 c0 = __ldg(reinterpret_cast<const float4*>(blk + o * 8));
-                    const float4 c1 = __ldg(reinterpret_cast<const float4*>(blk + o * 8 + 4));
+                    const float4 c0 = __ldg(blk + (o * 2 + 0) * 4);
+                    const float4 c1 = __ldg(blk + (o * 2 + 1) * 4);
                     const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                     float sa = 0.f, sb = 0.f;
 #pragma unroll
@@ -334,31 +372,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         cluster_arrive();             // my E has been read: the partner may send the next tile
 
         // ------------------------------------------------------ store ---
-        // thread -> (row, beta' pair); 32 loads of two bf16 (beta' = 2p, 2p+1) across the 32
-        // pencils of this CTA, repacked into two 64-byte runs of the output row.
-        {
-            const int row = tid >> 5, pidx = tid & 31;
+        // work item (row, p, u): beta' pair p = (2p, 2p+1), pencil quarter u = a_local >> 3.
+        // Eight word loads give the 8 pencils of the quarter for both beta'; each becomes a
+        // 16-byte piece of a 64-byte output run.  A warp covers one row, 8 pairs, 4 quarters,
+        // so each 16-byte store instruction writes 8 whole runs.
+#pragma unroll 1
+        for (int it = 0; it < 4; ++it) {
+            const int item = tid + kThreads * it;
+            const int row = item >> 7, pp = (item >> 2) & 31, u = item & 3;
             const int64_t grow = row0 + row;
             if (grow < p.rows) {
-                const int i2 = pidx >> 2, i3 = 2 * (pidx & 3);
-                uint32_t wv[32];
+                const int i2 = pp >> 2, i3 = 2 * (pp & 3);
+                uint32_t wv[8];
 #pragma unroll
-                for (int al = 0; al < 32; ++al)
-                    wv[al] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, al, i2, i3));
-                uint32_t run0[16], run1[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    run0[k] = __byte_perm(wv[2 * k], wv[2 * k + 1], 0x5410);
-                    run1[k] = __byte_perm(wv[2 * k], wv[2 * k + 1], 0x7632);
-                }
-                __nv_bfloat16* yrow = p.y + grow * p.ldy + 32 * r;
-                uint4* d0 = reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * i3));
-                uint4* d1 = reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * (i3 + 1)));
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    d0[k] = make_uint4(run0[4 * k], run0[4 * k + 1], run0[4 * k + 2], run0[4 * k + 3]);
-                    d1[k] = make_uint4(run1[4 * k], run1[4 * k + 1], run1[4 * k + 2], run1[4 * k + 3]);
-                }
+                for (int k = 0; k < 8; ++k)
+                    wv[k] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, 8 * u + k, i2, i3));
+                const uint4 r0 = make_uint4(__byte_perm(wv[0], wv[1], 0x5410), __byte_perm(wv[2], wv[3], 0x5410),
+                                            __byte_perm(wv[4], wv[5], 0x5410), __byte_perm(wv[6], wv[7], 0x5410));
+                const uint4 r1 = make_uint4(__byte_perm(wv[0], wv[1], 0x7632), __byte_perm(wv[2], wv[3], 0x7632),
+                                            __byte_perm(wv[4], wv[5], 0x7632), __byte_perm(wv[6], wv[7], 0x7632));
+                __nv_bfloat16* yrow = p.y + grow * p.ldy + 32 * r + 8 * u;
+                *reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * i3)) = r0;
+                *reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * (i3 + 1))) = r1;
             }
         }
         __syncthreads();              // O (= S) read before the next tile's phase A writes S
@@ -383,12 +418,32 @@ __global__ void pack_fragments_kernel(const float* __restrict__ blk, float2* __r
     out[gid] = make_float2(b[o * 8 + k0], b[o * 8 + k1]);
 }
 
+// Lane-interleaved copy of the blocks of a register stage, so that the four lanes
+// q = 0..3 of a quad, which work on blocks whose index differs by `qstride`, read
+// one contiguous 64-byte run per instruction:
+//   out[(((h * 2 + s) * 8 + o) * 2 + half) * 4 + q] = Blk_{c}[o][4 half .. 4 half + 3],
+//   c = base(h) + (q + 4 s) * qstride, with base(h) = 8h (stage 1: h = chunk) or h (stage 3: h = pencil).
+__global__ void pack_interleaved_kernel(const float* __restrict__ blk, float4* __restrict__ out, int nheads,
+                                        int head_mul, int qstride) {
+    const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= nheads * 128) return;
+    const int q = gid & 3, half = (gid >> 2) & 1, o = (gid >> 3) & 7, s = (gid >> 6) & 1, h = gid >> 7;
+    const int c = h * head_mul + (q + 4 * s) * qstride;
+    const float* b = blk + (size_t)c * 64 + o * 8 + 4 * half;
+    out[gid] = make_float4(b[0], b[1], b[2], b[3]);
+}
+
 struct FastState {
     float2* pk0 = nullptr;
     float2* pk2 = nullptr;
+    float4* pk1 = nullptr;
+    float4* pk3 = nullptr;
     int max_pairs = 0;
     bool ready = false;
 };
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
 
 bool is_d4096_radix8(const harp_plan_s* p) {
     if (p->desc.d != kD || p->desc.m != 4) return false;
@@ -404,15 +459,32 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
         fs = new FastState();
         p->fast = fs;
     }
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) == cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        cudaGetLastError();
+    });
+    if (!g_encode) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     const int nblocks = kD / 8;
-    if (cudaMalloc((void**)&fs->pk0, sizeof(float2) * nblocks * 32) != cudaSuccess ||
-        cudaMalloc((void**)&fs->pk2, sizeof(float2) * nblocks * 32) != cudaSuccess) {
+    if ((!fs->pk0 && cudaMalloc((void**)&fs->pk0, sizeof(float2) * nblocks * 32) != cudaSuccess) ||
+        (!fs->pk2 && cudaMalloc((void**)&fs->pk2, sizeof(float2) * nblocks * 32) != cudaSuccess) ||
+        (!fs->pk1 && cudaMalloc((void**)&fs->pk1, sizeof(float4) * nblocks * 16) != cudaSuccess) ||
+        (!fs->pk3 && cudaMalloc((void**)&fs->pk3, sizeof(float4) * nblocks * 16) != cudaSuccess)) {
         cudaGetLastError();
         return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the fragment tables failed");
     }
     const int threads = 256, grid = (nblocks * 32 + threads - 1) / threads;
-    pack_fragments_kernel<<<grid, threads, 0, stream>>>(p->d_blocks + p->desc.st[0].block_off, fs->pk0, nblocks, 1);
-    pack_fragments_kernel<<<grid, threads, 0, stream>>>(p->d_blocks + p->desc.st[2].block_off, fs->pk2, nblocks, 0);
+    const float* blocks = p->d_blocks;
+    pack_fragments_kernel<<<grid, threads, 0, stream>>>(blocks + p->desc.st[0].block_off, fs->pk0, nblocks, 1);
+    pack_fragments_kernel<<<grid, threads, 0, stream>>>(blocks + p->desc.st[2].block_off, fs->pk2, nblocks, 0);
+    // stage 1: block c = i0 + 8 beta, i0 = q + 4s;  stage 3: block c = a + 64 i2, i2 = q + 4s
+    pack_interleaved_kernel<<<(64 * 128 + threads - 1) / threads, threads, 0, stream>>>(
+        blocks + p->desc.st[1].block_off, fs->pk1, 64, 8, 1);
+    pack_interleaved_kernel<<<(64 * 128 + threads - 1) / threads, threads, 0, stream>>>(
+        blocks + p->desc.st[3].block_off, fs->pk3, 64, 1, 64);
     cudaError_t e = cudaFuncSetAttribute(harp_fast_d4096_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
@@ -440,29 +512,37 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               harp_dtype out_dtype) {
     if (!is_d4096_radix8(p) || in_dtype != HARP_BF16 || out_dtype != HARP_BF16 || dir != HARP_FORWARD)
         return HARP_ERR_UNSUPPORTED;
-    // 4-byte aligned input words, 16-byte aligned output runs
-    if (((uintptr_t)x & 3) || (ld_x & 1) || ((uintptr_t)y & 15) || (ld_y & 7)) return HARP_ERR_UNSUPPORTED;
-    if (rows < 32) return HARP_ERR_UNSUPPORTED;
+    // TMA input boxes need 16-byte aligned rows; output runs are 16-byte stores
+    if (((uintptr_t)x & 15) || (ld_x & 7) || ((uintptr_t)y & 15) || (ld_y & 7)) return HARP_ERR_UNSUPPORTED;
+    if (rows < 32 || rows > 0x7fffffffll) return HARP_ERR_UNSUPPORTED;
     cudaStream_t stream = (cudaStream_t)stream_;
     harp_status st = prepare(p, stream);
     if (st != HARP_OK) return st;
     FastState* fs = static_cast<FastState*>(p->fast);
     const int64_t ntiles = (rows + kTile - 1) / kTile;
-    if (ntiles > 0x7fffffff) return HARP_ERR_UNSUPPORTED;
     const int pairs = (int)std::min<int64_t>(fs->max_pairs, ntiles);
+
+    CUtensorMap tmap;
+    const cuuint64_t gdim[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)ld_x * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box,
+                           estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)cr));
+
     FastParams fp;
-    fp.x = reinterpret_cast<const uint32_t*>(x);
     fp.y = reinterpret_cast<__nv_bfloat16*>(y);
     fp.rows = rows;
-    fp.ldx_w = ld_x / 2;
     fp.ldy = ld_y;
     fp.ntiles = (int)ntiles;
     fp.pk0 = fs->pk0;
-    fp.blk1 = p->d_blocks + p->desc.st[1].block_off;
+    fp.pk1 = fs->pk1;
     fp.pk2 = fs->pk2;
-    fp.blk3 = p->d_blocks + p->desc.st[3].block_off;
+    fp.pk3 = fs->pk3;
     fp.status = p->d_status;
-    harp_fast_d4096_fwd_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(fp);
+    harp_fast_d4096_fwd_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_fast_d4096_fwd_kernel");
@@ -473,7 +553,9 @@ void fast_state_free(harp_plan_s* p) {
     FastState* fs = static_cast<FastState*>(p->fast);
     if (!fs) return;
     cudaFree(fs->pk0);
+    cudaFree(fs->pk1);
     cudaFree(fs->pk2);
+    cudaFree(fs->pk3);
     delete fs;
     p->fast = nullptr;
 }
