@@ -85,6 +85,67 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Two independent fp32 fused multiply-adds (round to nearest) on register pairs.
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ unsigned long long pair(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ float2 unpair(unsigned long long v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+
+// y[o] = sum_l B[o][l] x[l] for the 8 outputs of one block and two rows (A, B), with the
+// block read as 16 float4 = (B[2p][2k], B[2p+1][2k], B[2p][2k+1], B[2p+1][2k+1]) at
+// cf[(p * 4 + k) * 4] (p = output pair, k = input pair), four lanes apart.  Output pairs
+// (2p, 2p+1) accumulate in f32x2 registers; each row's inputs are duplicated once.
+__device__ __forceinline__ void block_matvec_2rows(const float4* __restrict__ cf, const float (&xa)[8],
+                                                   const float (&xb)[8], float (&ya)[8], float (&yb)[8]) {
+    unsigned long long da[8], db[8];
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+        da[l] = pair(xa[l], xa[l]);
+        db[l] = pair(xb[l], xb[l]);
+    }
+    float4 cur[4], nxt[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) cur[k] = __ldg(cf + k * 4);
+#pragma unroll
+    for (int op = 0; op < 4; ++op) {
+        if (op < 3) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) nxt[k] = __ldg(cf + ((op + 1) * 4 + k) * 4);
+        }
+        unsigned long long accA = 0ull, accB = 0ull;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const unsigned long long c0 = pair(cur[k].x, cur[k].y);   // (B[2op][2k],   B[2op+1][2k])
+            const unsigned long long c1 = pair(cur[k].z, cur[k].w);   // (B[2op][2k+1], B[2op+1][2k+1])
+            accA = ffma2(c0, da[2 * k], accA);
+            accB = ffma2(c0, db[2 * k], accB);
+            accA = ffma2(c1, da[2 * k + 1], accA);
+            accB = ffma2(c1, db[2 * k + 1], accB);
+        }
+        const float2 ra = unpair(accA), rb = unpair(accB);
+        ya[2 * op] = ra.x; ya[2 * op + 1] = ra.y;
+        yb[2 * op] = rb.x; yb[2 * op + 1] = rb.y;
+        if (op < 3) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
+        }
+    }
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -153,22 +214,23 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 
 // ------------------------------------------------------ shared layouts ---
 //
-// E[half][row][a_local][pos]: half = beta >> 5 (the CTA whose chunks produced it),
-// a_local = pencil index inside the owning CTA (a = 32 r + a_local), and
-// pos = (beta & 31) ^ swz(row, a_local) with swz = ((row & 7) << 2) | (a_local & 3).
-//  - phase A stores one scalar per lane with beta fixed, row = g (+8), a_local & 3 = q:
-//    banks (beta ^ (4g + q)) mod 32 are 32 distinct values.
-//  - phase B loads one scalar per lane with a_local fixed and beta = q + 8m (+4),
-//    row = g (+8): (q + 8m) ^ (4g + c) puts q in bits 0-1 and g in bits 2-4, so
-//    the 32 lanes again hit 32 distinct banks.
+// E[half][beta_local][row][pos]: half = beta >> 5 (the CTA whose chunks produced it),
+// beta_local = beta & 31, a_local = pencil index inside the owning CTA (a = 32 r + a_local)
+// and pos = a_local ^ swz(row, beta) with swz = ((row & 7) << 2) | (beta & 3).
+//  - phase A stores one scalar per lane with beta fixed, row = g (+8), a_local = q + 4s + 8o':
+//    a_local ^ (4g + c) has q ^ c in bits 0-1 and g ^ (s + 2o') in bits 2-4, 32 banks.
+//  - phase B loads one scalar per lane with a_local fixed, row = g (+8) and beta = q + 8m (+4),
+//    so beta & 3 = q: a_local ^ (4g + q) is a permutation of 0..31, 32 banks.
+// Each chunk's 16 x 32 block is contiguous (2 KB), so the part of it bound for the partner
+// CTA is sent with one bulk copy as soon as the warp has produced it.
 __device__ __forceinline__ int e_index(int half, int row, int a_local, int beta) {
-    const int swz = ((row & 7) << 2) | (a_local & 3);
-    return ((half * 16 + row) * 32 + a_local) * 32 + ((beta & 31) ^ swz);
+    const int swz = ((row & 7) << 2) | (beta & 3);
+    return ((half * 32 + (beta & 31)) * 16 + row) * 32 + (a_local ^ swz);
 }
 
 __device__ __forceinline__ int s_index(int row, int a_local, int beta) {
-    const int swz = ((row & 7) << 2) | (a_local & 3);
-    return (row * 32 + a_local) * 32 + ((beta & 31) ^ swz);
+    const int swz = ((row & 7) << 2) | (beta & 3);
+    return ((beta & 31) * 16 + row) * 32 + (a_local ^ swz);
 }
 
 // Output staging O[row][a_local][beta'] (bf16) with beta' = 8 i2 + i3, stored in 16-byte
@@ -218,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (tid == 0) mbar_init(bar, 1);
     if (lane == 0) mbar_init(xbar + warp, 1);
-    const uint32_t remote_e = map_to_rank(smem_u32(E + r * kSFloats), (uint32_t)(r ^ 1));
+    const uint32_t remote_e = map_to_rank(smem_u32(E + r * kSFloats), (uint32_t)(r ^ 1));   // partner's half r
     const uint32_t remote_bar = map_to_rank(smem_u32(bar), (uint32_t)(r ^ 1));
     cluster_arrive();
     cluster_wait();     // barriers initialised on both CTAs
@@ -234,6 +296,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int tile = pair; tile < p.ntiles; tile += npairs) {
         const int64_t row0 = (int64_t)tile * kTile;
         if (tid == 0) mbar_arrive_expect_tx(bar, kHalfBytes);
+        cluster_wait();               // the partner has finished reading its E (previous tile)
 
         // -------------------------------------------------- phase A ---
 #pragma unroll 1
@@ -250,10 +313,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stage 0 on tensor cores: group j = i1, slot q <-> i0 = 2q, slot q+4 <-> i0 = 2q+1;
             // output slot 2q <-> i0 = q, 2q+1 <-> i0 = q + 4.
             float z[8][4];
+            float2 bf[8];             // all eight B fragments in flight before the first mma
+#pragma unroll
+            for (int j = 0; j < 8; ++j) bf[j] = __ldg(p.pk0 + (size_t)(j + 8 * beta) * 32 + lane);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t a[4] = {w0[j] << 16, w1[j] << 16, w0[j] & 0xffff0000u, w1[j] & 0xffff0000u};
-                const float2 bb = __ldg(p.pk0 + (size_t)(j + 8 * beta) * 32 + lane);
+                const float2 bb = bf[j];
                 uint32_t bh0, bl0, bh1, bl1;
                 split_tf32(bb.x, bh0, bl0);
                 split_tf32(bb.y, bh1, bl1);
@@ -277,37 +343,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stage 1 in registers: this lane holds i1 = 0..7 of groups i0 = q + 4s for rows g, g+8
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
-                const float4* blk = p.pk1 + (size_t)((beta * 2 + s) * 8) * 8 + q;
+                float xa[8], xb[8], ya[8], yb[8];
+#pragma unroll
+                for (int l = 0; l < 8; ++l) {
+                    xa[l] = z[l][s];
+                    xb[l] = z[l][s + 2];
+                }
+                block_matvec_2rows(p.pk1 + (size_t)(beta * 2 + s) * 64 + q, xa, xb, ya, yb);
 #pragma unroll
                 for (int o = 0; o < 8; ++o) {
-                    const float4 c0 = __ldg(blk + (o * 2 + 0) * 4);
-                    const float4 c1 = __ldg(blk + (o * 2 + 1) * 4);
-                    const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    float yA = 0.f, yB = 0.f;
-#pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        yA = fmaf(cf[l], z[l][s], yA);
-                        yB = fmaf(cf[l], z[l][s + 2], yB);
-                    }
                     // coordinate (i0 = q + 4s, i1 = o, beta): pencil a_local = i0 + 8 (o & 3) of CTA o >> 2
                     const int a_local = (q + 4 * s) + 8 * (o & 3);
                     if ((o >> 2) == r) {
-                        E[e_index(r, g, a_local, beta)] = yA;
-                        E[e_index(r, g + 8, a_local, beta)] = yB;
+                        E[e_index(r, g, a_local, beta)] = ya[o];
+                        E[e_index(r, g + 8, a_local, beta)] = yb[o];
                     } else {
-                        S[s_index(g, a_local, beta)] = yA;
-                        S[s_index(g + 8, a_local, beta)] = yB;
+                        S[s_index(g, a_local, beta)] = ya[o];
+                        S[s_index(g + 8, a_local, beta)] = yb[o];
                     }
                 }
+            }
+            // this chunk's partner-bound 2 KB goes out now, overlapping the rest of phase A
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const int off = (beta & 31) * 16 * 32;
+                bulk_copy_to_cluster(remote_e + off * 4, S + off, 16 * 32 * 4, remote_bar);
             }
         }
 
         // --------------------------------------------------- exchange ---
-        fence_proxy_async_smem();     // S written through the generic proxy, read by the bulk copy
-        __syncthreads();
-        cluster_wait();               // the partner has finished reading its E
-        if (tid == 0) bulk_copy_to_cluster(remote_e, S, kHalfBytes, remote_bar);
-        if (!mbar_wait(bar, parity) && lane == 0) atomicExch(p.status, 1);
+        __syncthreads();              // local E writes of all warps
+        if (!mbar_wait(bar, parity) && lane == 0) atomicExch(p.status, 1);   // partner's 32 chunks
         parity ^= 1;
         cluster_arrive();             // both copies have landed: S may be reused
         cluster_wait();
@@ -320,6 +387,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stage 2 on tensor cores: group m = i3, slot q <-> i2 = q, slot q+4 <-> i2 = q + 4;
             // output slot 2q <-> i2 = q, 2q+1 <-> i2 = q + 4.
             float z2[8][4];
+            float2 bf[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) bf[m] = __ldg(p.pk2 + (size_t)(a + 64 * m) * 32 + lane);
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int half = m >> 2;
@@ -329,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 uint32_t ah[4], al[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) split_tf32(v[e], ah[e], al[e]);
-                const float2 bb = __ldg(p.pk2 + (size_t)(a + 64 * m) * 32 + lane);
+                const float2 bb = bf[m];
                 uint32_t bh0, bl0, bh1, bl1;
                 split_tf32(bb.x, bh0, bl0);
                 split_tf32(bb.y, bh1, bl1);
@@ -344,22 +414,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
                 const int i2 = q + 4 * s;
-                const float4* blk = p.pk3 + (size_t)((a * 2 + s) * 8) * 8 + q;
-                float yA[8], yB[8];
+                float xa[8], xb[8], yA[8], yB[8];
 #pragma unroll
-                for (int o = 0; o < 8; ++o) {
-                    const float4 c0 = __ldg(blk + (o * 2 + 0) * 4);
-                    const float4 c1 = __ldg(blk + (o * 2 + 1) * 4);
-                    const float cf[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    float sa = 0.f, sb = 0.f;
-#pragma unroll
-                    for (int l = 0; l < 8; ++l) {
-                        sa = fmaf(cf[l], z2[l][s], sa);
-                        sb = fmaf(cf[l], z2[l][s + 2], sb);
-                    }
-                    yA[o] = sa;
-                    yB[o] = sb;
+                for (int l = 0; l < 8; ++l) {
+                    xa[l] = z2[l][s];
+                    xb[l] = z2[l][s + 2];
                 }
+                block_matvec_2rows(p.pk3 + (size_t)(a * 2 + s) * 64 + q, xa, xb, yA, yB);
                 const uint4 pa = make_uint4(pack_bf16x2(yA[0], yA[1]), pack_bf16x2(yA[2], yA[3]),
                                             pack_bf16x2(yA[4], yA[5]), pack_bf16x2(yA[6], yA[7]));
                 const uint4 pb = make_uint4(pack_bf16x2(yB[0], yB[1]), pack_bf16x2(yB[2], yB[3]),
@@ -376,7 +437,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // Eight word loads give the 8 pencils of the quarter for both beta'; each becomes a
         // 16-byte piece of a 64-byte output run.  A warp covers one row, 8 pairs, 4 quarters,
         // so each 16-byte store instruction writes 8 whole runs.
-#pragma unroll 1
+#pragma unroll
         for (int it = 0; it < 4; ++it) {
             const int item = tid + kThreads * it;
             const int row = item >> 7, pp = (item >> 2) & 31, u = item & 3;
@@ -419,18 +480,20 @@ __global__ void pack_fragments_kernel(const float* __restrict__ blk, float2* __r
 }
 
 // Lane-interleaved copy of the blocks of a register stage, so that the four lanes
-// q = 0..3 of a quad, which work on blocks whose index differs by `qstride`, read
-// one contiguous 64-byte run per instruction:
-//   out[(((h * 2 + s) * 8 + o) * 2 + half) * 4 + q] = Blk_{c}[o][4 half .. 4 half + 3],
-//   c = base(h) + (q + 4 s) * qstride, with base(h) = 8h (stage 1: h = chunk) or h (stage 3: h = pencil).
+// q = 0..3 of a quad, which work on blocks whose index differs by `qstride`, read one
+// contiguous 64-byte run per instruction, and each float4 holds two output pairs:
+//   out[(((h * 2 + s) * 4 + p) * 4 + k) * 4 + q] =
+//       (B[2p][2k], B[2p+1][2k], B[2p][2k+1], B[2p+1][2k+1])   of block
+//   c = h * head_mul + (q + 4 s) * qstride   (stage 1: chunk h, c = 8h + i0;  stage 3: pencil h, c = h + 64 i2).
 __global__ void pack_interleaved_kernel(const float* __restrict__ blk, float4* __restrict__ out, int nheads,
                                         int head_mul, int qstride) {
     const int gid = blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= nheads * 128) return;
-    const int q = gid & 3, half = (gid >> 2) & 1, o = (gid >> 3) & 7, s = (gid >> 6) & 1, h = gid >> 7;
+    const int q = gid & 3, k = (gid >> 2) & 3, pr = (gid >> 4) & 3, s = (gid >> 6) & 1, h = gid >> 7;
     const int c = h * head_mul + (q + 4 * s) * qstride;
-    const float* b = blk + (size_t)c * 64 + o * 8 + 4 * half;
-    out[gid] = make_float4(b[0], b[1], b[2], b[3]);
+    const float* b = blk + (size_t)c * 64;
+    out[gid] = make_float4(b[(2 * pr) * 8 + 2 * k], b[(2 * pr + 1) * 8 + 2 * k], b[(2 * pr) * 8 + 2 * k + 1],
+                           b[(2 * pr + 1) * 8 + 2 * k + 1]);
 }
 
 struct FastState {
