@@ -13,14 +13,23 @@
 // with one 64 KB bulk copy (TMA engine, shared::cluster) completed on the
 // partner's mbarrier.
 //
-// Inner engine, per phase:
-//   * first stage: tensor cores, mma.sync m16n8k8 TF32 with the 16 tile rows as M,
-//     the 8 inputs of a group as K and its 8 outputs as N.  fp32 accuracy comes
-//     from splitting operands into TF32 hi + lo parts (round to nearest) and
-//     summing hi*hi + hi*lo + lo*hi; bf16 input is exact in TF32, so stage 0 needs
-//     only hi*hi + hi*lo.  Operand and output slots are permuted so that each lane
-//     ends up holding complete groups of the next stage.
-//   * second stage: plain fp32 FMA in each lane on the groups it already holds.
+// Inner engine: every stage runs on tensor cores, mma.sync m16n8k8 TF32 with the 16
+// tile rows as M, the 8 inputs of a group as K and its 8 outputs as N.  fp32 accuracy
+// comes from splitting operands into TF32 hi + lo parts and summing hi*hi + hi*lo +
+// lo*hi (bf16 input is exact in TF32, so stage 0 needs only hi*hi + hi*lo).
+//
+// Coefficients are stationary in tensor memory: each warp always works on the same
+// two chunks and two pencils, whose 64 blocks in mma B-fragment form are exactly
+// 128 words per lane, i.e. the warp's quarter of its TMEM lane quadrant.  They are
+// written once per launch and read with tcgen05.ld, so the coefficients cost no L2
+// traffic inside the row loop.
+//
+// Between the two stages of a phase the mma output (lane q holds two outputs of every
+// group) is turned into the next stage's operand (lane q holds two inputs of every
+// group) by a 4-lane butterfly: three shfl.xor rounds plus an XOR permutation by the
+// lane's quad index (two levels of selects).  The K slots of the second stage
+// therefore mean different inputs in different lanes; the packed B fragments
+// follow the same lane-dependent order.
 // Every shared-memory access pattern below is XOR-swizzled to be bank-conflict
 // free; the derivations are next to each index function.
 #include <cstdio>
@@ -45,17 +54,15 @@ constexpr int kHalfBytes = kSFloats * 4;     // 65536
 constexpr int kXBytes = 16 * 128;            // one 16-row x 64-column bf16 input box per warp
 constexpr int kXOffset = (kEFloats + kSFloats) * 4;          // 196608, 1024-aligned
 constexpr int kBarOffset = kXOffset + kWarps * kXBytes;      // 229376
-constexpr size_t kSmemBytes = (size_t)kBarOffset + 8 * (kWarps + 1) + 1024;   // + alignment slack
+constexpr size_t kSmemBytes = (size_t)kBarOffset + 8 * (kWarps + 1) + 16 + 1024;   // + TMEM slot, alignment slack
+constexpr int kTmemCols = 512;               // the SM's whole tensor memory: 128 columns per warp
 constexpr long long kWaitLimit = 1ll << 26;  // mbarrier polls before giving up
 
 struct FastParams {
     __nv_bfloat16* y;
     int64_t rows, ldy;       // ldy in elements
     int ntiles;
-    const float2* pk0;       // stage-0 B fragments, [block][lane]
-    const float4* pk1;       // stage-1 blocks, lane-interleaved (see pack_interleaved_kernel)
-    const float2* pk2;       // stage-2 B fragments
-    const float4* pk3;       // stage-3 blocks, lane-interleaved
+    const float4* frag;      // B fragments, [cta rank][warp][column / 4][lane] float4 (see pack kernel)
     int* status;
 };
 
@@ -71,10 +78,11 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
     return r;
 }
 
-// x = hi + lo with both parts TF32 (round to nearest): |x - hi - lo| <= 2^-22 |x|
+// x = hi + lo: hi is x rounded to TF32, lo = x - hi is exact in fp32 and the tensor
+// core reads its top 19 bits; |x - hi - lo_tf32| <= 2^-10 |lo| <= 2^-21 |x|.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
     hi = to_tf32(x);
-    lo = to_tf32(x - __uint_as_float(hi));
+    lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -83,67 +91,6 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Two independent fp32 fused multiply-adds (round to nearest) on register pairs.
-__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-__device__ __forceinline__ unsigned long long pair(float lo, float hi) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-__device__ __forceinline__ float2 unpair(unsigned long long v) {
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-    return r;
-}
-
-// y[o] = sum_l B[o][l] x[l] for the 8 outputs of one block and two rows (A, B), with the
-// block read as 16 float4 = (B[2p][2k], B[2p+1][2k], B[2p][2k+1], B[2p+1][2k+1]) at
-// cf[(p * 4 + k) * 4] (p = output pair, k = input pair), four lanes apart.  Output pairs
-// (2p, 2p+1) accumulate in f32x2 registers; each row's inputs are duplicated once.
-__device__ __forceinline__ void block_matvec_2rows(const float4* __restrict__ cf, const float (&xa)[8],
-                                                   const float (&xb)[8], float (&ya)[8], float (&yb)[8]) {
-    unsigned long long da[8], db[8];
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-        da[l] = pair(xa[l], xa[l]);
-        db[l] = pair(xb[l], xb[l]);
-    }
-    float4 cur[4], nxt[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) cur[k] = __ldg(cf + k * 4);
-#pragma unroll
-    for (int op = 0; op < 4; ++op) {
-        if (op < 3) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) nxt[k] = __ldg(cf + ((op + 1) * 4 + k) * 4);
-        }
-        unsigned long long accA = 0ull, accB = 0ull;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const unsigned long long c0 = pair(cur[k].x, cur[k].y);   // (B[2op][2k],   B[2op+1][2k])
-            const unsigned long long c1 = pair(cur[k].z, cur[k].w);   // (B[2op][2k+1], B[2op+1][2k+1])
-            accA = ffma2(c0, da[2 * k], accA);
-            accB = ffma2(c0, db[2 * k], accB);
-            accA = ffma2(c1, da[2 * k + 1], accA);
-            accB = ffma2(c1, db[2 * k + 1], accB);
-        }
-        const float2 ra = unpair(accA), rb = unpair(accB);
-        ya[2 * op] = ra.x; ya[2 * op + 1] = ra.y;
-        yb[2 * op] = rb.x; yb[2 * op + 1] = rb.y;
-        if (op < 3) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) cur[k] = nxt[k];
-        }
-    }
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -216,33 +163,34 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 //
 // E[half][beta_local][row][pos]: half = beta >> 5 (the CTA whose chunks produced it),
 // beta_local = beta & 31, a_local = pencil index inside the owning CTA (a = 32 r + a_local)
-// and pos = a_local ^ swz(row, beta) with swz = ((row & 7) << 2) | (beta & 3).
-//  - phase A stores one scalar per lane with beta fixed, row = g (+8), a_local = q + 4s + 8o':
-//    a_local ^ (4g + c) has q ^ c in bits 0-1 and g ^ (s + 2o') in bits 2-4, 32 banks.
-//  - phase B loads one scalar per lane with a_local fixed, row = g (+8) and beta = q + 8m (+4),
-//    so beta & 3 = q: a_local ^ (4g + q) is a permutation of 0..31, 32 banks.
+// and pos = a_local ^ swz(row, beta) with swz = (row & 7) | ((beta & 3) << 3).
+//  - phase A stores one scalar per lane with beta fixed, row = g (+8) and a_local = l + 8q:
+//    (l + 8q) ^ (g + 8c) has l ^ g in bits 0-2 and q ^ c in bits 3-4, 32 banks.
+//  - phase B loads one scalar per lane with a_local fixed, row = g (+8) and
+//    beta = q + 8m (+4), so beta & 3 = q: a_local ^ (g + 8q), 32 banks.
 // Each chunk's 16 x 32 block is contiguous (2 KB), so the part of it bound for the partner
 // CTA is sent with one bulk copy as soon as the warp has produced it.
 __device__ __forceinline__ int e_index(int half, int row, int a_local, int beta) {
-    const int swz = ((row & 7) << 2) | (beta & 3);
+    const int swz = (row & 7) | ((beta & 3) << 3);
     return ((half * 32 + (beta & 31)) * 16 + row) * 32 + (a_local ^ swz);
 }
 
 __device__ __forceinline__ int s_index(int row, int a_local, int beta) {
-    const int swz = ((row & 7) << 2) | (beta & 3);
+    const int swz = (row & 7) | ((beta & 3) << 3);
     return ((beta & 31) * 16 + row) * 32 + (a_local ^ swz);
 }
 
-// Output staging O[row][a_local][beta'] (bf16) with beta' = 8 i2 + i3, stored in 16-byte
-// chunks indexed by i2 ^ h, h = 2 ((a_local >> 3) & 3) ^ 4 (row & 1).
-//  - phase B stores a 16-byte chunk per lane (a_local fixed, i2 = q + 4s, rows 2k and 2k+1
-//    in a quarter-warp): the row bit moves the chunk to the other half, 8 distinct chunks.
-//  - the store phase loads one word per thread with the row fixed, 8 consecutive beta'
-//    pairs and the 4 pencil quarters u = a_local >> 3: chunks (p >> 2) ^ 2u are 8 distinct
-//    values and p & 3 selects the word, 32 distinct banks.
-__device__ __forceinline__ int o_byte(int row, int a_local, int i2, int i3) {
-    const int chunk = i2 ^ ((((a_local >> 3) & 3) << 1) ^ ((row & 1) << 2));
-    return ((row * 32 + a_local) * 64 + chunk * 8 + i3) * 2;
+// Output staging O[row][a_local][beta] (bf16), stored in 16-byte chunks of 8 beta values
+// (chunk = i3 = beta >> 3, inside the chunk i2 = beta & 7) at chunk position
+// i3 ^ h, h = (row & 1) ^ (2 ((a_local >> 3) & 3)).
+//  - phase B stores one chunk per lane (a_local fixed, i3 = 2q + e, rows 2k and 2k+1 in a
+//    quarter-warp): the row bit moves the chunk to the other parity, 8 distinct chunks.
+//  - the store phase loads one word (two beta) per thread with the row fixed, 8
+//    consecutive beta pairs and the 4 pencil quarters u: chunks (pp >> 2) ^ 2u ^ c are 8
+//    distinct values and pp & 3 selects the word, 32 banks.
+__device__ __forceinline__ int o_byte(int row, int a_local, int beta) {
+    const int chunk = (beta >> 3) ^ ((row & 1) ^ (((a_local >> 3) & 3) << 1));
+    return ((row * 32 + a_local) * 64 + chunk * 8 + (beta & 7)) * 2;
 }
 
 // Input staging: TMA writes a 16 x 128-byte box with the 128-byte swizzle, i.e. the
@@ -255,6 +203,121 @@ __device__ __forceinline__ int x_byte(int row, int j, int q) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------- tensor memory ---
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ----------------------------------------------------- stage helpers ---
+
+// One stage of 8 groups on tensor cores from fp32 operands: d[l] = A[l] * B_l with the
+// A fragments split into hi + lo and the B fragments (two fp32 words per group, from
+// TMEM) split likewise; three products per group.
+__device__ __forceinline__ void mma_stage_f32(const float (&a)[8][4], const uint32_t (&bw)[16], float (&d)[8][4]) {
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_tf32(a[l][e], ah[e], al[e]);
+        uint32_t bh0, bl0, bh1, bl1;
+        split_tf32(__uint_as_float(bw[2 * l]), bh0, bl0);
+        split_tf32(__uint_as_float(bw[2 * l + 1]), bh1, bl1);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_tf32(acc, ah, bh0, bh1);
+        mma_tf32(acc, ah, bl0, bl1);
+        mma_tf32(acc, al, bh0, bh1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d[l][e] = acc[e];
+    }
+}
+
+__device__ __forceinline__ void cswap(bool p, float& x, float& y) {
+    const float a = p ? y : x;
+    const float b = p ? x : y;
+    x = a;
+    y = b;
+}
+
+// 4-lane butterfly between the two stages of a phase.
+// In:  z[j][e], the mma output of group j (e = s + 2h: output slot s of row half h), where
+//      output slot s of lane q is next-stage group c + 4s with c = q.
+// Out: a[l][e'], the A fragment of next-stage group l = c + 4s (e' = h + 2t), whose K slot t
+//      holds input j = (q ^ c) + 4t: round delta brings j = delta + 4t from lane q ^ delta.
+__device__ __forceinline__ void quad_butterfly(const float (&z)[8][4], int q, float (&a)[8][4]) {
+    float rr[4][2][2][2];   // [delta][t][s][h]
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                rr[0][t][s][h] = z[4 * t][s + 2 * h];
+#pragma unroll
+                for (int dl = 1; dl < 4; ++dl)
+                    rr[dl][t][s][h] = __shfl_xor_sync(0xffffffffu, z[dl + 4 * t][s + 2 * h], dl);
+            }
+    // rr[delta] came from lane q ^ delta; reorder so that rr[c] comes from lane c
+    const bool b0 = (q & 1) != 0, b1 = (q & 2) != 0;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                cswap(b0, rr[0][t][s][h], rr[1][t][s][h]);
+                cswap(b0, rr[2][t][s][h], rr[3][t][s][h]);
+                cswap(b1, rr[0][t][s][h], rr[2][t][s][h]);
+                cswap(b1, rr[1][t][s][h], rr[3][t][s][h]);
+            }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            a[c + 4 * s][0] = rr[c][0][s][0];
+            a[c + 4 * s][1] = rr[c][0][s][1];
+            a[c + 4 * s][2] = rr[c][1][s][0];
+            a[c + 4 * s][3] = rr[c][1][s][1];
+        }
 }
 
 // ------------------------------------------------------------- kernel ---
@@ -270,6 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     unsigned char* X = base + kXOffset;
     uint64_t* xbar = reinterpret_cast<uint64_t*>(base + kBarOffset);   // one per warp
     uint64_t* bar = xbar + kWarps;                                      // exchange
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -278,13 +342,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     unsigned char* Xw = X + warp * kXBytes;
 
+    // tensor memory: the whole 512 columns; warp w uses lanes 32 (w & 3).., columns 128 (w >> 2)..
+    if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
     if (tid == 0) mbar_init(bar, 1);
     if (lane == 0) mbar_init(xbar + warp, 1);
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    const uint32_t taddr = *tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + 128u * (uint32_t)(warp >> 2);
+    {
+        // this warp's 128 fragment columns: [slot (2 chunks, 2 pencils)][stage][group][word]
+        const float4* src = p.frag + ((size_t)(r * kWarps + warp) * 32) * 32 + lane;
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+            uint32_t v[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 f = __ldg(src + (c16 * 4 + k) * 32);
+                v[4 * k] = __float_as_uint(f.x);
+                v[4 * k + 1] = __float_as_uint(f.y);
+                v[4 * k + 2] = __float_as_uint(f.z);
+                v[4 * k + 3] = __float_as_uint(f.w);
+            }
+            tmem_st16(taddr + 16u * c16, v);
+        }
+        tmem_wait_st();
+    }
+
     const uint32_t remote_e = map_to_rank(smem_u32(E + r * kSFloats), (uint32_t)(r ^ 1));   // partner's half r
     const uint32_t remote_bar = map_to_rank(smem_u32(bar), (uint32_t)(r ^ 1));
     cluster_arrive();
     cluster_wait();     // barriers initialised on both CTAs
-    cluster_arrive();   // "my E may be written": matched by the wait before the first send
+    cluster_arrive();   // "my E may be written": matched by the wait at the top of the first tile
 
     // first input box of this warp: tile `pair`, task 0
     if (lane == 0 && pair < p.ntiles) {
@@ -302,6 +391,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int task = 0; task < 2; ++task) {
             const int beta = 32 * r + 2 * warp + task;
+            uint32_t bw[16];
+            tmem_ld16(taddr + 32u * task, bw);          // stage-0 fragments of this chunk
             if (!mbar_wait(xbar + warp, xparity) && lane == 0) atomicExch(p.status, 1);
             xparity ^= 1;
             uint32_t w0[8], w1[8];
@@ -310,19 +401,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 w0[j] = *reinterpret_cast<const uint32_t*>(Xw + x_byte(g, j, q));
                 w1[j] = *reinterpret_cast<const uint32_t*>(Xw + x_byte(g + 8, j, q));
             }
-            // stage 0 on tensor cores: group j = i1, slot q <-> i0 = 2q, slot q+4 <-> i0 = 2q+1;
+            tmem_wait_ld();
+            // stage 0: group j = i1, slot q <-> i0 = 2q, slot q+4 <-> i0 = 2q+1;
             // output slot 2q <-> i0 = q, 2q+1 <-> i0 = q + 4.
             float z[8][4];
-            float2 bf[8];             // all eight B fragments in flight before the first mma
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bf[j] = __ldg(p.pk0 + (size_t)(j + 8 * beta) * 32 + lane);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t a[4] = {w0[j] << 16, w1[j] << 16, w0[j] & 0xffff0000u, w1[j] & 0xffff0000u};
-                const float2 bb = bf[j];
                 uint32_t bh0, bl0, bh1, bl1;
-                split_tf32(bb.x, bh0, bl0);
-                split_tf32(bb.y, bh1, bl1);
+                split_tf32(__uint_as_float(bw[2 * j]), bh0, bl0);
+                split_tf32(__uint_as_float(bw[2 * j + 1]), bh1, bl1);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_tf32(d, a, bh0, bh1);
                 mma_tf32(d, a, bl0, bl1);
@@ -340,26 +428,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tma_load_2d(Xw, &tmap_x, 64 * (32 * r + 2 * warp + (task ^ 1)), ntile * kTile, xbar + warp);
                 }
             }
-            // stage 1 in registers: this lane holds i1 = 0..7 of groups i0 = q + 4s for rows g, g+8
+            tmem_ld16(taddr + 32u * task + 16u, bw);    // stage-1 fragments
+            float a1[8][4];
+            quad_butterfly(z, q, a1);
+            tmem_wait_ld();
+            // stage 1: group l = i0; output slot 2q <-> i1 = q (pencils of CTA 0),
+            // 2q+1 <-> i1 = q + 4 (pencils of CTA 1); both are pencil a_local = l + 8q there.
+            float y1[8][4];
+            mma_stage_f32(a1, bw, y1);
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                float xa[8], xb[8], ya[8], yb[8];
+            for (int l = 0; l < 8; ++l) {
+                const int a_local = l + 8 * q;
 #pragma unroll
-                for (int l = 0; l < 8; ++l) {
-                    xa[l] = z[l][s];
-                    xb[l] = z[l][s + 2];
-                }
-                block_matvec_2rows(p.pk1 + (size_t)(beta * 2 + s) * 64 + q, xa, xb, ya, yb);
-#pragma unroll
-                for (int o = 0; o < 8; ++o) {
-                    // coordinate (i0 = q + 4s, i1 = o, beta): pencil a_local = i0 + 8 (o & 3) of CTA o >> 2
-                    const int a_local = (q + 4 * s) + 8 * (o & 3);
-                    if ((o >> 2) == r) {
-                        E[e_index(r, g, a_local, beta)] = ya[o];
-                        E[e_index(r, g + 8, a_local, beta)] = yb[o];
+                for (int hh = 0; hh < 2; ++hh) {   // hh = destination CTA
+                    const float va = y1[l][hh], vb = y1[l][hh + 2];
+                    if (hh == r) {
+                        E[e_index(r, g, a_local, beta)] = va;
+                        E[e_index(r, g + 8, a_local, beta)] = vb;
                     } else {
-                        S[s_index(g, a_local, beta)] = ya[o];
-                        S[s_index(g + 8, a_local, beta)] = yb[o];
+                        S[s_index(g, a_local, beta)] = va;
+                        S[s_index(g + 8, a_local, beta)] = vb;
                     }
                 }
             }
@@ -376,65 +464,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncthreads();              // local E writes of all warps
         if (!mbar_wait(bar, parity) && lane == 0) atomicExch(p.status, 1);   // partner's 32 chunks
         parity ^= 1;
-        cluster_arrive();             // both copies have landed: S may be reused
+        cluster_arrive();             // both sides' copies have landed: S may be reused
         cluster_wait();
 
         // --------------------------------------------------- phase B ---
 #pragma unroll 1
         for (int task = 0; task < 2; ++task) {
             const int a_local = 2 * warp + task;
-            const int a = 32 * r + a_local;
-            // stage 2 on tensor cores: group m = i3, slot q <-> i2 = q, slot q+4 <-> i2 = q + 4;
+            uint32_t bw[16];
+            tmem_ld16(taddr + 32u * (2 + task), bw);    // stage-2 fragments of this pencil
+            // stage 2: group m = i3, slot q <-> i2 = q, slot q+4 <-> i2 = q + 4;
             // output slot 2q <-> i2 = q, 2q+1 <-> i2 = q + 4.
-            float z2[8][4];
-            float2 bf[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) bf[m] = __ldg(p.pk2 + (size_t)(a + 64 * m) * 32 + lane);
+            float v2[8][4];
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int half = m >> 2;
                 const int b0 = q + 8 * m, b1 = q + 4 + 8 * m;
-                const float v[4] = {E[e_index(half, g, a_local, b0)], E[e_index(half, g + 8, a_local, b0)],
-                                    E[e_index(half, g, a_local, b1)], E[e_index(half, g + 8, a_local, b1)]};
-                uint32_t ah[4], al[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) split_tf32(v[e], ah[e], al[e]);
-                const float2 bb = bf[m];
-                uint32_t bh0, bl0, bh1, bl1;
-                split_tf32(bb.x, bh0, bl0);
-                split_tf32(bb.y, bh1, bl1);
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_tf32(d, ah, bh0, bh1);
-                mma_tf32(d, ah, bl0, bl1);
-                mma_tf32(d, al, bh0, bh1);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) z2[m][e] = d[e];
+                v2[m][0] = E[e_index(half, g, a_local, b0)];
+                v2[m][1] = E[e_index(half, g + 8, a_local, b0)];
+                v2[m][2] = E[e_index(half, g, a_local, b1)];
+                v2[m][3] = E[e_index(half, g + 8, a_local, b1)];
             }
-            // stage 3 in registers: groups i2 = q + 4s, inputs i3 = 0..7
+            tmem_wait_ld();
+            float z2[8][4];
+            mma_stage_f32(v2, bw, z2);
+            tmem_ld16(taddr + 32u * (2 + task) + 16u, bw);   // stage-3 fragments
+            float a3[8][4];
+            quad_butterfly(z2, q, a3);
+            tmem_wait_ld();
+            // stage 3: group l = i2; output slot 2q <-> i3 = 2q, 2q+1 <-> i3 = 2q + 1
+            float y3[8][4];
+            mma_stage_f32(a3, bw, y3);
+            // bf16 runs of 8 consecutive beta (i2 = 0..7) for i3 = 2q + e, rows g and g + 8
 #pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int i2 = q + 4 * s;
-                float xa[8], xb[8], yA[8], yB[8];
+            for (int e = 0; e < 2; ++e) {
 #pragma unroll
-                for (int l = 0; l < 8; ++l) {
-                    xa[l] = z2[l][s];
-                    xb[l] = z2[l][s + 2];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c = e + 2 * hh;
+                    const uint4 pk = make_uint4(pack_bf16x2(y3[0][c], y3[1][c]), pack_bf16x2(y3[2][c], y3[3][c]),
+                                                pack_bf16x2(y3[4][c], y3[5][c]), pack_bf16x2(y3[6][c], y3[7][c]));
+                    *reinterpret_cast<uint4*>(O + o_byte(g + 8 * hh, a_local, 8 * (2 * q + e))) = pk;
                 }
-                block_matvec_2rows(p.pk3 + (size_t)(a * 2 + s) * 64 + q, xa, xb, yA, yB);
-                const uint4 pa = make_uint4(pack_bf16x2(yA[0], yA[1]), pack_bf16x2(yA[2], yA[3]),
-                                            pack_bf16x2(yA[4], yA[5]), pack_bf16x2(yA[6], yA[7]));
-                const uint4 pb = make_uint4(pack_bf16x2(yB[0], yB[1]), pack_bf16x2(yB[2], yB[3]),
-                                            pack_bf16x2(yB[4], yB[5]), pack_bf16x2(yB[6], yB[7]));
-                *reinterpret_cast<uint4*>(O + o_byte(g, a_local, i2, 0)) = pa;
-                *reinterpret_cast<uint4*>(O + o_byte(g + 8, a_local, i2, 0)) = pb;
             }
         }
         __syncthreads();
         cluster_arrive();             // my E has been read: the partner may send the next tile
 
         // ------------------------------------------------------ store ---
-        // work item (row, p, u): beta' pair p = (2p, 2p+1), pencil quarter u = a_local >> 3.
-        // Eight word loads give the 8 pencils of the quarter for both beta'; each becomes a
+        // work item (row, pp, u): beta pair (2pp, 2pp+1), pencil quarter u = a_local >> 3.
+        // Eight word loads give the 8 pencils of the quarter for both beta; each becomes a
         // 16-byte piece of a 64-byte output run.  A warp covers one row, 8 pairs, 4 quarters,
         // so each 16-byte store instruction writes 8 whole runs.
 #pragma unroll
@@ -443,64 +521,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int row = item >> 7, pp = (item >> 2) & 31, u = item & 3;
             const int64_t grow = row0 + row;
             if (grow < p.rows) {
-                const int i2 = pp >> 2, i3 = 2 * (pp & 3);
                 uint32_t wv[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    wv[k] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, 8 * u + k, i2, i3));
+                    wv[k] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, 8 * u + k, 2 * pp));
                 const uint4 r0 = make_uint4(__byte_perm(wv[0], wv[1], 0x5410), __byte_perm(wv[2], wv[3], 0x5410),
                                             __byte_perm(wv[4], wv[5], 0x5410), __byte_perm(wv[6], wv[7], 0x5410));
                 const uint4 r1 = make_uint4(__byte_perm(wv[0], wv[1], 0x7632), __byte_perm(wv[2], wv[3], 0x7632),
                                             __byte_perm(wv[4], wv[5], 0x7632), __byte_perm(wv[6], wv[7], 0x7632));
                 __nv_bfloat16* yrow = p.y + grow * p.ldy + 32 * r + 8 * u;
-                *reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * i3)) = r0;
-                *reinterpret_cast<uint4*>(yrow + 64 * (i2 + 8 * (i3 + 1))) = r1;
+                *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp)) = r0;
+                *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp + 1)) = r1;
             }
         }
         __syncthreads();              // O (= S) read before the next tile's phase A writes S
     }
     cluster_wait();                   // matches the last arrive; no bulk copy is in flight
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    if (warp == 0) tmem_dealloc(*tmem_slot, kTmemCols);
 }
 
-// B fragments of a block for mma.m16n8k8 (lane L = 4 g + q):
-//   b0 = B[q][g], b1 = B[q + 4][g] with B[k][n] = Blk[out(n)][in(k)],
-//   out(n) = n / 2 for even n, n / 2 + 4 for odd n,
-//   stage 0: in(q) = 2q, in(q + 4) = 2q + 1;   stage 2: in(k) = k.
-__global__ void pack_fragments_kernel(const float* __restrict__ blk, float2* __restrict__ out, int nblocks,
-                                      int interleaved_inputs) {
-    const int gid = blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= nblocks * 32) return;
-    const int c = gid >> 5, L = gid & 31;
+// B fragments for mma.m16n8k8, packed per (CTA rank r, warp w, lane L = 4g + q) into
+// 128 columns: column = slot * 32 + stage * 16 + group * 2 + word, where slots 0, 1 are
+// the chunks beta = 32r + 2w + slot (stages 0, 1) and slots 2, 3 the pencils
+// a = 32r + 2w + slot - 2 (stages 2, 3).  Word k of group n is B[k-th K slot][g] =
+// Blk[out(g)][in]:
+//   out(g) = g / 2 (even g), g / 2 + 4 (odd g) for stages 0-2; out(g) = g for stage 3;
+//   stage 0, block j + 8 beta:   in = 2q + k
+//   stage 1, block l + 8 beta:   in = (q ^ (l & 3)) + 4k
+//   stage 2, block a + 64 m:     in = q + 4k
+//   stage 3, block a + 64 l:     in = (q ^ (l & 3)) + 4k
+// Stored as float4 over 4 consecutive columns: frag[((r * 16 + w) * 32 + col / 4) * 32 + L].
+__global__ void pack_fragments_kernel(const float* __restrict__ b0, const float* __restrict__ b1,
+                                      const float* __restrict__ b2, const float* __restrict__ b3,
+                                      float* __restrict__ frag) {
+    const int gid = blockIdx.x * blockDim.x + threadIdx.x;   // one float per thread
+    if (gid >= 2 * kWarps * 128 * 32) return;
+    const int comp = gid & 3;
+    const int L = (gid >> 2) & 31;
+    const int col4 = (gid >> 7) & 31;
+    const int w = (gid >> 12) & 15;
+    const int r = gid >> 16;
+    const int col = col4 * 4 + comp;
+    const int slot = col >> 5, stage = (col >> 4) & 1, grp = (col >> 1) & 7, k = col & 1;
     const int g = L >> 2, q = L & 3;
-    const int o = (g & 1) ? (g >> 1) + 4 : (g >> 1);
-    const int k0 = interleaved_inputs ? 2 * q : q;
-    const int k1 = interleaved_inputs ? 2 * q + 1 : q + 4;
-    const float* b = blk + (size_t)c * 64;
-    out[gid] = make_float2(b[o * 8 + k0], b[o * 8 + k1]);
-}
-
-// Lane-interleaved copy of the blocks of a register stage, so that the four lanes
-// q = 0..3 of a quad, which work on blocks whose index differs by `qstride`, read one
-// contiguous 64-byte run per instruction, and each float4 holds two output pairs:
-//   out[(((h * 2 + s) * 4 + p) * 4 + k) * 4 + q] =
-//       (B[2p][2k], B[2p+1][2k], B[2p][2k+1], B[2p+1][2k+1])   of block
-//   c = h * head_mul + (q + 4 s) * qstride   (stage 1: chunk h, c = 8h + i0;  stage 3: pencil h, c = h + 64 i2).
-__global__ void pack_interleaved_kernel(const float* __restrict__ blk, float4* __restrict__ out, int nheads,
-                                        int head_mul, int qstride) {
-    const int gid = blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= nheads * 128) return;
-    const int q = gid & 3, k = (gid >> 2) & 3, pr = (gid >> 4) & 3, s = (gid >> 6) & 1, h = gid >> 7;
-    const int c = h * head_mul + (q + 4 * s) * qstride;
-    const float* b = blk + (size_t)c * 64;
-    out[gid] = make_float4(b[(2 * pr) * 8 + 2 * k], b[(2 * pr + 1) * 8 + 2 * k], b[(2 * pr) * 8 + 2 * k + 1],
-                           b[(2 * pr + 1) * 8 + 2 * k + 1]);
+    const int pn = (g & 1) ? (g >> 1) + 4 : (g >> 1);
+    float v;
+    if (slot < 2) {
+        const int beta = 32 * r + 2 * w + slot;
+        if (stage == 0) v = b0[(size_t)(grp + 8 * beta) * 64 + pn * 8 + 2 * q + k];
+        else            v = b1[(size_t)(grp + 8 * beta) * 64 + pn * 8 + ((q ^ (grp & 3)) + 4 * k)];
+    } else {
+        const int a = 32 * r + 2 * w + slot - 2;
+        if (stage == 0) v = b2[(size_t)(a + 64 * grp) * 64 + pn * 8 + q + 4 * k];
+        else            v = b3[(size_t)(a + 64 * grp) * 64 + g * 8 + ((q ^ (grp & 3)) + 4 * k)];
+    }
+    frag[gid] = v;
 }
 
 struct FastState {
-    float2* pk0 = nullptr;
-    float2* pk2 = nullptr;
-    float4* pk1 = nullptr;
-    float4* pk3 = nullptr;
+    float* frag = nullptr;
     int max_pairs = 0;
     bool ready = false;
 };
@@ -531,23 +613,15 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
         cudaGetLastError();
     });
     if (!g_encode) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-    const int nblocks = kD / 8;
-    if ((!fs->pk0 && cudaMalloc((void**)&fs->pk0, sizeof(float2) * nblocks * 32) != cudaSuccess) ||
-        (!fs->pk2 && cudaMalloc((void**)&fs->pk2, sizeof(float2) * nblocks * 32) != cudaSuccess) ||
-        (!fs->pk1 && cudaMalloc((void**)&fs->pk1, sizeof(float4) * nblocks * 16) != cudaSuccess) ||
-        (!fs->pk3 && cudaMalloc((void**)&fs->pk3, sizeof(float4) * nblocks * 16) != cudaSuccess)) {
+    const int nfloat = 2 * kWarps * 128 * 32;
+    if (!fs->frag && cudaMalloc((void**)&fs->frag, sizeof(float) * nfloat) != cudaSuccess) {
         cudaGetLastError();
-        return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the fragment tables failed");
+        return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the fragment table failed");
     }
-    const int threads = 256, grid = (nblocks * 32 + threads - 1) / threads;
     const float* blocks = p->d_blocks;
-    pack_fragments_kernel<<<grid, threads, 0, stream>>>(blocks + p->desc.st[0].block_off, fs->pk0, nblocks, 1);
-    pack_fragments_kernel<<<grid, threads, 0, stream>>>(blocks + p->desc.st[2].block_off, fs->pk2, nblocks, 0);
-    // stage 1: block c = i0 + 8 beta, i0 = q + 4s;  stage 3: block c = a + 64 i2, i2 = q + 4s
-    pack_interleaved_kernel<<<(64 * 128 + threads - 1) / threads, threads, 0, stream>>>(
-        blocks + p->desc.st[1].block_off, fs->pk1, 64, 8, 1);
-    pack_interleaved_kernel<<<(64 * 128 + threads - 1) / threads, threads, 0, stream>>>(
-        blocks + p->desc.st[3].block_off, fs->pk3, 64, 1, 64);
+    pack_fragments_kernel<<<(nfloat + 255) / 256, 256, 0, stream>>>(
+        blocks + p->desc.st[0].block_off, blocks + p->desc.st[1].block_off, blocks + p->desc.st[2].block_off,
+        blocks + p->desc.st[3].block_off, fs->frag);
     cudaError_t e = cudaFuncSetAttribute(harp_fast_d4096_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
@@ -600,10 +674,7 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     fp.rows = rows;
     fp.ldy = ld_y;
     fp.ntiles = (int)ntiles;
-    fp.pk0 = fs->pk0;
-    fp.pk1 = fs->pk1;
-    fp.pk2 = fs->pk2;
-    fp.pk3 = fs->pk3;
+    fp.frag = reinterpret_cast<const float4*>(fs->frag);
     fp.status = p->d_status;
     harp_fast_d4096_fwd_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp);
     cudaError_t e = cudaGetLastError();
@@ -615,10 +686,7 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
 void fast_state_free(harp_plan_s* p) {
     FastState* fs = static_cast<FastState*>(p->fast);
     if (!fs) return;
-    cudaFree(fs->pk0);
-    cudaFree(fs->pk1);
-    cudaFree(fs->pk2);
-    cudaFree(fs->pk3);
+    cudaFree(fs->frag);
     delete fs;
     p->fast = nullptr;
 }
