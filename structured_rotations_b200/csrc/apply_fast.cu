@@ -329,6 +329,34 @@ __device__ __forceinline__ void quad_butterfly(const float (&z)[8][4], int q, fl
         }
 }
 
+// Output row `row` of one tile, stored by one warp: item (pp, u) = beta pair (2pp, 2pp+1)
+// and pencil quarter u = a_local >> 3, four items per lane.  Eight word loads give the 8
+// pencils of the quarter for both beta; each becomes a 16-byte piece of a 64-byte output
+// run, so each 16-byte store instruction writes 8 whole runs.  Row w of O occupies exactly
+// the bytes of S that warp w writes next (its two chunks' 2 KB blocks), so no other warp
+// has to wait for these loads.
+__device__ __forceinline__ void store_row(const unsigned char* O, const FastParams& p, int64_t row0, int row,
+                                          int r, int lane) {
+    const int64_t grow = row0 + row;
+    if (grow >= p.rows) return;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int item = lane + 32 * it;
+        const int pp = item >> 2, u = item & 3;
+        uint32_t wv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            wv[k] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, 8 * u + k, 2 * pp));
+        const uint4 r0 = make_uint4(__byte_perm(wv[0], wv[1], 0x5410), __byte_perm(wv[2], wv[3], 0x5410),
+                                    __byte_perm(wv[4], wv[5], 0x5410), __byte_perm(wv[6], wv[7], 0x5410));
+        const uint4 r1 = make_uint4(__byte_perm(wv[0], wv[1], 0x7632), __byte_perm(wv[2], wv[3], 0x7632),
+                                    __byte_perm(wv[4], wv[5], 0x7632), __byte_perm(wv[6], wv[7], 0x7632));
+        __nv_bfloat16* yrow = p.y + grow * p.ldy + 32 * r + 8 * u;
+        *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp)) = r0;
+        *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp + 1)) = r1;
+    }
+}
+
 // ------------------------------------------------------------- kernel ---
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -392,11 +420,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tma_load_2d(Xw, &tmap_x, 64 * (32 * r + 2 * warp), pair * kTile, xbar + warp);
     }
     uint32_t xparity = 0, parity = 0;
+    int64_t prev_row0 = -1;           // tile whose output still sits in O
 
     for (int tile = pair; tile < p.ntiles; tile += npairs) {
         const int64_t row0 = (int64_t)tile * kTile;
         if (tid == 0) mbar_arrive_expect_tx(bar, kHalfBytes);
-        cluster_wait();               // the partner has finished reading its E (previous tile)
 
         // -------------------------------------------------- phase A ---
 #pragma unroll 1
@@ -446,6 +474,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // 2q+1 <-> i1 = q + 4 (pencils of CTA 1); both are pencil a_local = l + 8q there.
             float y1[8][4];
             mma_stage_f32(a1, bw, z2, y1);
+            if (task == 0) {
+                // row `warp` of the previous tile's output leaves O, which aliases the part
+                // of S this warp is about to write
+                if (prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
+                __syncwarp();
+                cluster_wait();       // the partner has finished reading its E (previous tile)
+            }
 #pragma unroll
             for (int l = 0; l < 8; ++l) {
                 const int a_local = l + 8 * q;
@@ -474,8 +509,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncthreads();              // local E writes of all warps
         if (!mbar_wait(bar, parity) && lane == 0) atomicExch(p.status, 1);   // partner's 32 chunks
         parity ^= 1;
-        cluster_arrive();             // both sides' copies have landed: S may be reused
-        cluster_wait();
+        cluster_arrive();             // the partner's copies have landed: its S may be reused
 
         // --------------------------------------------------- phase B ---
 #pragma unroll 1
@@ -505,6 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stage 3: group l = i2; output slot 2q <-> i3 = 2q, 2q+1 <-> i3 = 2q + 1
             float y3[8][4];
             mma_stage_f32(a3, bw, z2, y3);
+            if (task == 0) cluster_wait();   // my copies have landed too: O (= S) may be written
             // bf16 runs of 8 consecutive beta (i2 = 0..7) for i3 = 2q + e, rows g and g + 8
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -520,32 +555,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncthreads();
         cluster_arrive();             // my E has been read: the partner may send the next tile
 
-        // ------------------------------------------------------ store ---
-        // work item (row, pp, u): beta pair (2pp, 2pp+1), pencil quarter u = a_local >> 3.
-        // Eight word loads give the 8 pencils of the quarter for both beta; each becomes a
-        // 16-byte piece of a 64-byte output run.  A warp covers one row, 8 pairs, 4 quarters,
-        // so each 16-byte store instruction writes 8 whole runs.
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-            const int item = tid + kThreads * it;
-            const int row = item >> 7, pp = (item >> 2) & 31, u = item & 3;
-            const int64_t grow = row0 + row;
-            if (grow < p.rows) {
-                uint32_t wv[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    wv[k] = *reinterpret_cast<const uint32_t*>(O + o_byte(row, 8 * u + k, 2 * pp));
-                const uint4 r0 = make_uint4(__byte_perm(wv[0], wv[1], 0x5410), __byte_perm(wv[2], wv[3], 0x5410),
-                                            __byte_perm(wv[4], wv[5], 0x5410), __byte_perm(wv[6], wv[7], 0x5410));
-                const uint4 r1 = make_uint4(__byte_perm(wv[0], wv[1], 0x7632), __byte_perm(wv[2], wv[3], 0x7632),
-                                            __byte_perm(wv[4], wv[5], 0x7632), __byte_perm(wv[6], wv[7], 0x7632));
-                __nv_bfloat16* yrow = p.y + grow * p.ldy + 32 * r + 8 * u;
-                *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp)) = r0;
-                *reinterpret_cast<uint4*>(yrow + 64 * (2 * pp + 1)) = r1;
-            }
-        }
-        __syncthreads();              // O (= S) read before the next tile's phase A writes S
+        prev_row0 = row0;             // its output is stored during the next tile's first task
     }
+    if (prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
     cluster_wait();                   // matches the last arrive; no bulk copy is in flight
     tmem_fence_before_sync();
     __syncthreads();
