@@ -24,13 +24,36 @@ harp_status check_device(const harp_plan_s* p) {
     return HARP_OK;
 }
 
-// 0 = auto, 1 = simple only, 2 = fast only (fail if the shape has no fast kernel)
+// HARP_KERNEL selects the row kernel: unset = the fastest one that covers the shape
+// (specialized, then tiled, then simple); "simple", "tiled" or "fast" (specialized)
+// force one and fail with HARP_ERR_UNSUPPORTED if it does not cover the shape.
+enum { kAuto = 0, kSimple = 1, kFast = 2, kTiled = 3 };
+
 int kernel_choice() {
     const char* v = std::getenv("HARP_KERNEL");
-    if (!v) return 0;
-    if (!std::strcmp(v, "simple")) return 1;
-    if (!std::strcmp(v, "fast")) return 2;
-    return 0;
+    if (!v) return kAuto;
+    if (!std::strcmp(v, "simple")) return kSimple;
+    if (!std::strcmp(v, "fast")) return kFast;
+    if (!std::strcmp(v, "tiled")) return kTiled;
+    return kAuto;
+}
+
+// The row kernels in order of preference.
+harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x, int64_t ld_y,
+                     harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir, void* stream) {
+    const int choice = kernel_choice();
+    harp_status st;
+    if (choice == kAuto || choice == kFast) {
+        st = launch_apply_fast(p, x, y, rows, ld_x, ld_y, in_dtype, dir, stream, out_dtype);
+        if (st != HARP_ERR_UNSUPPORTED || choice == kFast) return st;
+        harp_clear_error();
+    }
+    if (choice == kAuto || choice == kTiled) {
+        st = launch_apply_tiled(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
+        if (st != HARP_ERR_UNSUPPORTED || choice == kTiled) return st;
+        harp_clear_error();
+    }
+    return launch_apply_simple(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
 }
 
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
@@ -62,13 +85,7 @@ extern "C" harp_status harp_apply(harp_plan_t p, const void* x, void* y, int64_t
     } else if (ranges_overlap(x, ((rows - 1) * ld_x + d) * es, y, ((rows - 1) * ld_y + d) * es)) {
         return harp_fail(HARP_ERR_INVALID_ARG, "x and y overlap without being equal");
     }
-    const int choice = kernel_choice();
-    if (choice != 1) {
-        st = launch_apply_fast(p, x, y, rows, ld_x, ld_y, dtype, dir, stream, dtype);
-        if (st != HARP_ERR_UNSUPPORTED || choice == 2) return st;
-        harp_clear_error();
-    }
-    return launch_apply_simple(p, x, y, rows, ld_x, ld_y, dtype, dtype, dir, stream);
+    return run_rows(p, x, y, rows, ld_x, ld_y, dtype, dtype, dir, stream);
 }
 
 extern "C" size_t harp_two_sided_workspace_bytes(int64_t n_out, int64_t n_in) {
@@ -106,20 +123,12 @@ extern "C" harp_status harp_apply_two_sided(harp_plan_t pu, harp_plan_t pv, cons
     float* ws1 = (float*)workspace;
     float* ws2 = (float*)((char*)workspace + harp_two_sided_workspace_bytes(n_out, n_in) / 2);
     // rows of W: w_r <- T_V^T w_r (fp32 out)
-    st = launch_apply_fast(pv, W, ws1, n_out, ld, n_in, dtype, HARP_INVERSE, stream, HARP_F32);
-    if (st == HARP_ERR_UNSUPPORTED) {
-        harp_clear_error();
-        st = launch_apply_simple(pv, W, ws1, n_out, ld, n_in, dtype, HARP_F32, HARP_INVERSE, stream);
-    }
+    st = run_rows(pv, W, ws1, n_out, ld, n_in, dtype, HARP_F32, HARP_INVERSE, stream);
     if (st != HARP_OK) return st;
     if ((st = launch_transpose(ws1, ws2, n_out, n_in, n_in, n_out, HARP_F32, HARP_F32, stream)) != HARP_OK)
         return st;
     // columns of W (rows of W^T): col <- T_U^T col
-    st = launch_apply_fast(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_INVERSE, stream, HARP_F32);
-    if (st == HARP_ERR_UNSUPPORTED) {
-        harp_clear_error();
-        st = launch_apply_simple(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_F32, HARP_INVERSE, stream);
-    }
+    st = run_rows(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_F32, HARP_INVERSE, stream);
     if (st != HARP_OK) return st;
     return launch_transpose(ws2, W_out, n_in, n_out, n_out, ld, HARP_F32, dtype, stream);
 }

@@ -71,3 +71,9 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               int64_t ld_x, int64_t ld_y, harp_dtype in_dtype, harp_dir dir,
                               void* stream, harp_dtype out_dtype);
 void fast_state_free(harp_plan_s* p);
+
+// General tiled row kernel (apply_tiled.cu): radices 2..8, d % 8 == 0, 16-byte aligned
+// rows.  Returns HARP_ERR_UNSUPPORTED for other shapes.
+harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
+                               int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
+                               void* stream);

@@ -1,0 +1,136 @@
+"""GPU parity of the general tiled row kernel (forced with HARP_KERNEL=tiled) against
+the float64 oracle: every workload schedule in both directions, schedules that use
+each radix 2..8 (so every radix-set instantiation runs), ragged tiles, padded
+leading dimensions, in-place calls; and its fallback rules."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from oracle import harp_oracle as O
+import workloads as W
+import structured_rotations_b200 as H
+from structured_rotations_b200 import harp as HB
+from tests._parity import check_bf16, check_f32
+from tests.test_parity_gpu import plans, to_dev, to_host, decode, check, run
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture
+def tiled(monkeypatch):
+    monkeypatch.setenv("HARP_KERNEL", "tiled")
+    yield
+    assert H.last_kernel() == "harp_tiled_kernel"
+
+
+@pytest.mark.parametrize("name,direction", [
+    ("c1", "forward"), ("c1", "inverse"), ("c1b", "forward"),
+    ("c2", "forward"), ("c2", "inverse"), ("c3", "forward"), ("c3", "inverse"),
+    ("c5", "forward"), ("c5", "inverse")])
+@pytest.mark.parametrize("rows", [1, 5, 37, 300])
+def test_workloads_full_compare(tiled, name, direction, rows):
+    gp, tr = plans(name)
+    enc = W.draw_encoded(W.get(name), 0, rows)
+    out = run(gp, enc, direction)
+    check(out, tr.apply(decode(enc), direction), decode(enc), f"tiled {name} {direction} rows={rows}")
+
+
+def _plan_pair(schedule, seed):
+    d = int(np.prod(schedule))
+    theta = W.draw_theta(O.theta_count(schedule), 0.05, seed)
+    gp = H.Plan(d, schedule, theta=theta, sign_seed=seed + 1)
+    gp.materialize()
+    return gp, O.Transform(O.make_plan(d, schedule, theta, sign_seed=seed + 1))
+
+
+OTHER_SCHEDULES = [(5, 2, 8), (7, 8), (8, 5), (4, 4, 4), (3, 8), (6, 4), (2, 2, 2, 2),
+                   (8, 7, 2), (2, 8, 8), (8, 8, 2, 3)]
+
+
+@pytest.mark.parametrize("schedule", OTHER_SCHEDULES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_other_radices(tiled, schedule, dtype):
+    gp, tr = _plan_pair(schedule, 900 + sum(schedule))
+    d = int(np.prod(schedule))
+    rng = np.random.default_rng(d)
+    # enough elements that the share of near-zero outputs held to the fp32 bound
+    # (rather than one bf16 step) is a meaningful statistic
+    x = rng.standard_normal((max(53, 65536 // d), d))
+    enc = W.encode_bf16(x) if dtype == "bf16" else x.astype(np.float32)
+    xf = decode(enc)
+    for direction in ("forward", "inverse"):
+        out = run(gp, enc, direction)
+        check(out, tr.apply(xf, direction), xf, f"tiled {schedule} {dtype} {direction}")
+
+
+@pytest.mark.parametrize("name", ["c1", "c3", "c5"])
+def test_same_bits_as_the_simple_kernel(monkeypatch, name):
+    """Both kernels sum each output as fma(B[k][l], x_l, acc) over l = 0..b-1 from 0, so
+    their fp32 results agree bit for bit."""
+    gp, _ = plans(name)
+    enc = W.draw_encoded(W.get(name), 0, 41)
+    outs = {}
+    for kernel in ("tiled", "simple"):
+        monkeypatch.setenv("HARP_KERNEL", kernel)
+        for direction in ("forward", "inverse"):
+            x = to_dev(enc)
+            if x.dtype == torch.bfloat16:
+                x = x.float()
+            outs[kernel, direction] = to_host(gp.apply(x, direction=direction))
+    for direction in ("forward", "inverse"):
+        np.testing.assert_array_equal(outs["tiled", direction], outs["simple", direction])
+
+
+@pytest.mark.parametrize("name", ["c3", "c5", "c1"])
+def test_in_place(tiled, name):
+    gp, tr = plans(name)
+    enc = W.draw_encoded(W.get(name), 0, 23)
+    x = to_dev(enc)
+    gp.apply(x, x, direction="inverse")
+    torch.cuda.synchronize()
+    check(to_host(x), tr.inverse(decode(enc)), decode(enc), f"tiled {name} in place")
+
+
+@pytest.mark.parametrize("name,pad", [("c3", 8), ("c5", 64), ("c1", 4)])
+def test_padded_rows_and_guard_bands(tiled, name, pad):
+    gp, tr = plans(name)
+    w = W.get(name)
+    rows, d = 29, w.d
+    ld = d + pad
+    enc = W.draw_encoded(w, 0, rows)
+    canary = 0x7FC1 if enc.dtype == np.uint16 else np.float32(-123.25)
+    buf_x = np.full(rows * ld + 64, canary, dtype=enc.dtype)
+    buf_x[:rows * ld].reshape(rows, ld)[:, :d] = enc
+    buf_y = np.full(rows * ld + 64, canary, dtype=enc.dtype)
+    tx, ty = to_dev(buf_x), to_dev(buf_y)
+    gp.apply(tx[:rows * ld].view(rows, ld)[:, :d], ty[:rows * ld].view(rows, ld)[:, :d])
+    torch.cuda.synchronize()
+    got = to_host(ty)
+    body = got[:rows * ld].reshape(rows, ld)
+    check(np.ascontiguousarray(body[:, :d]), tr.forward(decode(enc)), decode(enc), f"tiled {name} ld={ld}")
+    assert np.all(body[:, d:] == canary) and np.all(got[rows * ld:] == canary)
+    np.testing.assert_array_equal(to_host(tx), buf_x)
+
+
+def test_shapes_outside_the_tiled_kernel_fall_back(monkeypatch):
+    gp, tr = _plan_pair((3, 3), 77)            # d = 9 is not a multiple of 8
+    x = np.random.default_rng(1).standard_normal((40, 9)).astype(np.float32)
+    monkeypatch.delenv("HARP_KERNEL", raising=False)
+    out = run(gp, x, "forward")
+    assert H.last_kernel() == "apply_simple_kernel"
+    check(out, tr.forward(x.astype(np.float64)), x.astype(np.float64), "d=9 fallback")
+    monkeypatch.setenv("HARP_KERNEL", "tiled")
+    with pytest.raises(HB.HarpError) as e:
+        gp.apply(to_dev(x))
+    assert e.value.status == HB.HARP_ERR_UNSUPPORTED
+
+
+def test_default_dispatch_takes_the_tiled_kernel_for_c3_and_c5(monkeypatch):
+    monkeypatch.delenv("HARP_KERNEL", raising=False)
+    for name, direction in (("c3", "forward"), ("c5", "inverse"), ("c2", "inverse")):
+        gp, _ = plans(name)
+        run(gp, W.draw_encoded(W.get(name), 0, 64), direction)
+        assert H.last_kernel() == "harp_tiled_kernel", name
+        gp.device_status()
