@@ -49,23 +49,35 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     while (which < kNumMasks && (kMasks[which] & mask) != mask) ++which;
     if (which == kNumMasks) return HARP_ERR_UNSUPPORTED;
 
-    // Rows per tile: fp32 tile plus a staging area for the next tile's raw rows when two
-    // or more rows fit that way, else the fp32 tile alone (loads then do not overlap).
-    const int64_t per_row_staged = d * (4 + es_in);
-    const int64_t per_row = d * 4;
+    // Rows per tile R = V Q: Q sub-tiles of V = 4 rows (fp32, 16 d bytes each), plus a
+    // staging area for the next tile's raw rows unless staging would halve Q; sub-tiles of
+    // one row when not even one 4-row sub-tile fits.
     const int64_t budget = kSmemOptIn - 64;
-    int64_t R = std::min<int64_t>(kMaxTileRows, budget / per_row_staged);
-    int staged = 1;
-    if (R < 2) {
-        R = std::min<int64_t>(kMaxTileRows, budget / per_row);
+    const int64_t q_staged = std::min<int64_t>(budget / (4 * d * (4 + es_in)), kMaxTileRows / 4);
+    const int64_t q_plain = std::min<int64_t>(budget / (16 * d), kMaxTileRows / 4);
+    int V = 4, staged = 1;
+    int64_t Q = q_staged;
+    if (q_plain >= 2 * q_staged) {
+        Q = q_plain;
         staged = 0;
     }
-    if (R < 1) return HARP_ERR_UNSUPPORTED;
-    R = std::min<int64_t>(R, rows);
+    if (Q < 1) {
+        V = 1;
+        Q = std::min<int64_t>(budget / (d * (4 + es_in)), kMaxTileRows);
+        staged = 1;
+        if (Q < 2) {
+            Q = std::min<int64_t>(budget / (d * 4), kMaxTileRows);
+            staged = 0;
+        }
+        if (Q < 1 || !has_row_major_kernel(kMasks[which])) return HARP_ERR_UNSUPPORTED;
+    }
+    Q = std::min<int64_t>(Q, (rows + V - 1) / V);
+    const int64_t R = V * Q;
 
     TiledParams tp;
     tp.pd = p->desc;
-    tp.blocks = p->d_blocks;
+    tp.lanes = p->d_blocks_lanes;
+    for (int t = 0; t < HARP_MAX_STAGES; ++t) tp.lane_off[t] = p->lane_off[t];
     tp.x = x;
     tp.y = y;
     tp.rows = rows;
@@ -74,19 +86,19 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.ntiles = (rows + R - 1) / R;
     tp.R = (int)R;
     tp.staged = staged;
-    tp.swz = (d % 32 == 0) ? 0x18 : 0;
+    tp.mask = (d % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
-    const size_t smem = (size_t)(staged ? per_row_staged : per_row) * R + 16;
+    const size_t smem = (size_t)R * d * 4 + (staged ? (size_t)R * d * es_in : 0) + 16;
     const int grid = (int)std::min<int64_t>(tp.ntiles, sm_count());
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;
     cudaError_t e;
     if (in_dtype == HARP_BF16 && out_dtype == HARP_BF16)
-        e = harp_tiled_launch_bf16(which, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16(which, V, inv, tp, smem, grid, s);
     else if (in_dtype == HARP_F32)
-        e = harp_tiled_launch_f32(which, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_f32(which, V, inv, tp, smem, grid, s);
     else
-        e = harp_tiled_launch_bf16_f32(which, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16_f32(which, V, inv, tp, smem, grid, s);
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_tiled_kernel");
     return HARP_OK;

@@ -7,7 +7,7 @@
 // fp32 across all m stages, so HBM is read once and written once.  While the stages
 // of tile k run, the bulk-copy engine (cp.async.bulk, completed on an mbarrier)
 // brings the raw rows of the CTA's next tile into a staging area, so loads overlap
-// the arithmetic.
+// the arithmetic (when the staging area fits next to the tile).
 //
 // Stage t: each thread takes whole groups {lo + s_t (k + b_t hi)} (block c = lo +
 // s_t hi), holds the block B_{t,c} (b_t x b_t fp32, plain FMA arithmetic) in
@@ -16,13 +16,16 @@
 // while the current one is applied.  The inverse runs the stages backwards with
 // B^T (the signs S are folded into stage 0's blocks, so B_0^T also applies S last).
 //
-// Shared-memory layout of a row: element i lives at word i ^ ((i >> 3) & 0x18)
-// (bits 6-7 of i XORed into bits 3-4; identity if d is not a multiple of 32).
-//  - stride 1 (stage 0 of a radix-8 schedule): a thread reads 8 consecutive words,
-//    the XOR keeps 8-aligned runs contiguous, so two 16-byte accesses per row.
-//  - stride 8: lanes c = lo + 8 hi read lo + 8k + 64 hi; the four lanes sharing lo
-//    have four different hi & 3, so the XOR puts them in four different banks.
-//  - stride >= 32: 32 consecutive lo per warp, one bank each.
+// Shared-memory layout: the tile is a stack of sub-tiles of V = 4 rows; inside one,
+// coordinate i holds the 4 rows' values as one 16-byte quad at quad index
+// slot(i) = i ^ ((i >> 3) & 7).  A thread therefore moves 4 rows with one 16-byte access
+// and keeps 4 independent accumulators per output.  The XOR spreads the quads a warp
+// touches over the 8 bank groups a quarter-warp's 16-byte accesses need:
+//  - stride 1 (lanes c read 8c + k): quad index mod 8 = k ^ (c & 7), 8 distinct;
+//  - stride 8 (lanes c = lo + 8 hi read lo + 8k + 64 hi): mod 8 = lo ^ k, 8 distinct;
+//  - stride >= 64 (consecutive lo): 8 consecutive quads permuted, 8 distinct.
+// When even one 4-row sub-tile of fp32 does not fit (d > 14524), sub-tiles are single
+// rows (V = 1) with word index i ^ ((i >> 3) & 0x18).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,14 +42,15 @@ constexpr long long kWaitLimit = 1ll << 26;   // mbarrier polls before giving up
 
 struct TiledParams {
     PlanDesc pd;
-    const float* blocks;
+    const float* lanes;                      // lane-interleaved blocks
+    int64_t lane_off[HARP_MAX_STAGES];       // per stage, in floats
     const void* x;
     void* y;
     int64_t rows, ld_x, ld_y;   // in elements
     int64_t ntiles;
-    int R;                      // rows per tile
+    int R;                      // rows per tile (a multiple of the sub-tile height V)
     int staged;                 // 1: rows of the next tile arrive by bulk copy
-    int swz;                    // 0x18 when d % 32 == 0, else 0
+    int mask;                   // V = 1 swizzle: 0x18 when d % 32 == 0, else 0
     int* status;
 };
 
@@ -97,7 +101,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 // ------------------------------------------------------------ helpers ---
 
-__device__ __forceinline__ int swz(int i, int mask) { return i ^ ((i >> 3) & mask); }
+// Vector of the V rows of one sub-tile at one coordinate.
+template <int V> struct VecOf;
+template <> struct VecOf<4> { using T = float4; };
+template <> struct VecOf<1> { using T = float; };
+
+// Position of coordinate i inside a sub-tile, in units of VecOf<V> (layout notes above).
+template <int V>
+__device__ __forceinline__ int slot(int i, int mask) {
+    if constexpr (V == 4) return i ^ ((i >> 3) & 7);
+    else return i ^ ((i >> 3) & mask);
+}
 
 // 8 consecutive elements <-> 8 floats
 __device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
@@ -128,109 +142,97 @@ __device__ __forceinline__ void store8(__nv_bfloat16* dst, const float (&v)[8]) 
     *(uint4*)dst = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Block B_{t,c}: b*b floats, row-major [output k][input l].
+// Block B_{t,c} (b*b floats, row-major [output k][input l]) from the stage's
+// lane-interleaved copy: lanes holding 32 consecutive c read contiguous memory.
 template <int B>
-__device__ __forceinline__ void load_block(float (&w)[B * B], const float* __restrict__ src, bool vec) {
+__device__ __forceinline__ void load_block(float (&w)[B * B], const float* __restrict__ stage, int c) {
+    const int group = c >> 5, lane = c & 31;
     if constexpr ((B * B) % 4 == 0) {
-        if (vec) {
+        const float4* src = (const float4*)stage + (size_t)group * (B * B / 4) * 32 + lane;
 #pragma unroll
-            for (int q = 0; q < B * B / 4; ++q) {
-                const float4 v = __ldg((const float4*)src + q);
-                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-            }
-            return;
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < B * B; ++q) w[q] = __ldg(src + q);
-}
-
-// One group of one row: y = B x (forward) or y = B^T x (inverse), in place.
-template <int B, bool INV>
-__device__ __forceinline__ void group_row(float* __restrict__ row, const int (&pos)[B], bool contig,
-                                          const float (&w)[B * B]) {
-    float xv[B];
-    if constexpr (B % 4 == 0) {
-        if (contig) {
-#pragma unroll
-            for (int q = 0; q < B / 4; ++q) {
-                const float4 v = *(const float4*)(row + pos[4 * q]);
-                xv[4 * q] = v.x; xv[4 * q + 1] = v.y; xv[4 * q + 2] = v.z; xv[4 * q + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int l = 0; l < B; ++l) xv[l] = row[pos[l]];
+        for (int q = 0; q < B * B / 4; ++q) {
+            const float4 v = __ldg(src + q * 32);
+            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
         }
     } else {
+        const float* src = stage + (size_t)group * (B * B) * 32 + lane;
 #pragma unroll
-        for (int l = 0; l < B; ++l) xv[l] = row[pos[l]];
+        for (int e = 0; e < B * B; ++e) w[e] = __ldg(src + e * 32);
     }
-    float yv[B];
-#pragma unroll
-    for (int k = 0; k < B; ++k) {
-        float acc = 0.0f;
-#pragma unroll
-        for (int l = 0; l < B; ++l) acc = fmaf(INV ? w[l * B + k] : w[k * B + l], xv[l], acc);
-        yv[k] = acc;
-    }
-    if constexpr (B % 4 == 0) {
-        if (contig) {
-#pragma unroll
-            for (int q = 0; q < B / 4; ++q)
-                *(float4*)(row + pos[4 * q]) = make_float4(yv[4 * q], yv[4 * q + 1], yv[4 * q + 2], yv[4 * q + 3]);
-            return;
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < B; ++k) row[pos[k]] = yv[k];
 }
 
-// Item = (block c, row group g): the rows g, g + G, ... of the tile.
-template <int B, bool INV>
-__device__ __forceinline__ void apply_item(float* data, int d, int nr, int G, int nb, int s, int swzmask,
-                                           int item, const float (&w)[B * B]) {
+__device__ __forceinline__ void fma_v(float4& acc, float w, const float4& x) {
+    acc.x = fmaf(w, x.x, acc.x);
+    acc.y = fmaf(w, x.y, acc.y);
+    acc.z = fmaf(w, x.z, acc.z);
+    acc.w = fmaf(w, x.w, acc.w);
+}
+__device__ __forceinline__ void fma_v(float& acc, float w, const float& x) { acc = fmaf(w, x, acc); }
+__device__ __forceinline__ void zero_v(float4& v) { v = make_float4(0.f, 0.f, 0.f, 0.f); }
+__device__ __forceinline__ void zero_v(float& v) { v = 0.f; }
+
+// One group in one sub-tile (V rows at once): y = B x (forward) or B^T x (inverse), in
+// place.  Each output is summed as fma(B[k][l], x_l, acc) over l = 0..b-1 from zero.
+template <int B, bool INV, typename VT>
+__device__ __forceinline__ void group_vec(VT* __restrict__ st, const int (&pos)[B], const float (&w)[B * B]) {
+    VT xv[B];
+#pragma unroll
+    for (int l = 0; l < B; ++l) xv[l] = st[pos[l]];
+    VT yv[B];
+#pragma unroll
+    for (int k = 0; k < B; ++k) {
+        zero_v(yv[k]);
+#pragma unroll
+        for (int l = 0; l < B; ++l) fma_v(yv[k], INV ? w[l * B + k] : w[k * B + l], xv[l]);
+    }
+#pragma unroll
+    for (int k = 0; k < B; ++k) st[pos[k]] = yv[k];
+}
+
+// Item = (block c, sub-tile group g): the sub-tiles g, g + G, ... of the tile.
+template <int B, bool INV, int V>
+__device__ __forceinline__ void apply_item(typename VecOf<V>::T* tile, int d, int qv, int G, int nb, int s,
+                                           int mask, int item, const float (&w)[B * B]) {
     const int c = item % nb;
     const int g = item / nb;
     const int lo = c % s, hi = c / s;
     const int base = lo + s * B * hi;
     int pos[B];
 #pragma unroll
-    for (int k = 0; k < B; ++k) pos[k] = swz(base + s * k, swzmask);
-    const bool contig = (s == 1);
-    for (int r = g; r < nr; r += G) group_row<B, INV>(data + r * d, pos, contig, w);
+    for (int k = 0; k < B; ++k) pos[k] = slot<V>(base + s * k, mask);
+    for (int q = g; q < qv; q += G) group_vec<B, INV>(tile + q * d, pos, w);
 }
 
 // All items of one stage; the coefficients of the thread's next item are loaded while
 // the current one is applied.
-template <int B, bool INV>
-__device__ __forceinline__ void run_stage(const StageDesc& sd, const float* __restrict__ blocks, float* data,
-                                          int d, int nr, int swzmask) {
+template <int B, bool INV, int V>
+__device__ __forceinline__ void run_stage(const StageDesc& sd, const float* __restrict__ sb,
+                                          typename VecOf<V>::T* tile, int d, int qv, int mask) {
     const int nb = d / B;
     const int s = (int)sd.s;
-    // Row groups: enough items to keep every thread busy, evenly spread.
+    // Sub-tile groups: split the tile's sub-tiles over more items only while too few
+    // items would leave a fifth or more of the threads' slots empty.
     int G = 1;
-    while (G < nr && G < 8) {
+    while (G < qv) {
         const int items = nb * G;
         const int per = (items + kThreads - 1) / kThreads;
-        if (per * kThreads <= items + items / 8) break;   // >= ~89% of the threads' slots used
+        if (per * kThreads * 4 <= items * 5) break;
         ++G;
     }
     const int items = nb * G;
-    const float* sb = blocks + sd.block_off;
-    const bool vec = (sd.block_off & 3) == 0;
     int j = threadIdx.x;
     if (j >= items) return;
     float wa[B * B], wb[B * B];
-    load_block<B>(wa, sb + (j % nb) * (B * B), vec);
+    load_block<B>(wa, sb, j % nb);
     while (true) {
         int jn = j + kThreads;
-        if (jn < items) load_block<B>(wb, sb + (jn % nb) * (B * B), vec);
-        apply_item<B, INV>(data, d, nr, G, nb, s, swzmask, j, wa);
+        if (jn < items) load_block<B>(wb, sb, jn % nb);
+        apply_item<B, INV, V>(tile, d, qv, G, nb, s, mask, j, wa);
         if (jn >= items) break;
         j = jn;
         jn = j + kThreads;
-        if (jn < items) load_block<B>(wa, sb + (jn % nb) * (B * B), vec);
-        apply_item<B, INV>(data, d, nr, G, nb, s, swzmask, j, wb);
+        if (jn < items) load_block<B>(wa, sb, jn % nb);
+        apply_item<B, INV, V>(tile, d, qv, G, nb, s, mask, j, wb);
         if (jn >= items) break;
         j = jn;
     }
@@ -248,29 +250,99 @@ __device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, u
     for (int r = 0; r < nr; ++r) bulk_load(stage_buf + (size_t)r * row_bytes, x + (row0 + r) * p.ld_x, row_bytes, bar);
 }
 
-template <typename TIn, typename TOut, bool INV, int MASK>
+// Rows -> sub-tiles.  V = 4: a thread takes 8 consecutive coordinates of the 4 rows of a
+// sub-tile and writes them as 8 quads.  V = 1: 8 consecutive coordinates of one row, two
+// 16-byte stores (the XOR keeps 8-aligned runs contiguous).  Rows past the end of the
+// batch are zero.
+template <int V, typename TIn>
+__device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int nr, const TIn* src, int64_t ld,
+                                          int mask) {
+    const int d8 = d / 8;
+    for (int q = 0; V * q < nr; ++q)
+        for (int j = threadIdx.x; j < d8; j += kThreads) {
+            if constexpr (V == 4) {
+                float v[4][8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (4 * q + e < nr) {
+                        load8(src + (4 * q + e) * ld + 8 * j, v[e]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) v[e][k] = 0.0f;
+                    }
+                }
+                float4* st = tile + q * d;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) st[slot<4>(8 * j + k, mask)] = make_float4(v[0][k], v[1][k], v[2][k], v[3][k]);
+            } else {
+                float v[8];
+                load8(src + q * ld + 8 * j, v);
+                store8(tile + q * d + slot<1>(8 * j, mask), v);
+            }
+        }
+}
+
+template <int V, typename TOut>
+__device__ __forceinline__ void drain_tile(const typename VecOf<V>::T* tile, int d, int nr, TOut* dst, int64_t ld,
+                                           int mask) {
+    const int d8 = d / 8;
+    for (int q = 0; V * q < nr; ++q)
+        for (int j = threadIdx.x; j < d8; j += kThreads) {
+            if constexpr (V == 4) {
+                const float4* st = tile + q * d;
+                float4 v4[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v4[k] = st[slot<4>(8 * j + k, mask)];
+                float v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = v4[k].x;
+                store8(dst + (4 * q) * ld + 8 * j, v);
+                if (4 * q + 1 < nr) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) v[k] = v4[k].y;
+                    store8(dst + (4 * q + 1) * ld + 8 * j, v);
+                }
+                if (4 * q + 2 < nr) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) v[k] = v4[k].z;
+                    store8(dst + (4 * q + 2) * ld + 8 * j, v);
+                }
+                if (4 * q + 3 < nr) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) v[k] = v4[k].w;
+                    store8(dst + (4 * q + 3) * ld + 8 * j, v);
+                }
+            } else {
+                float v[8];
+                load8(tile + q * d + slot<1>(8 * j, mask), v);
+                store8(dst + q * ld + 8 * j, v);
+            }
+        }
+}
+
+template <typename TIn, typename TOut, bool INV, int MASK, int V>
 __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_constant__ TiledParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    using VT = typename VecOf<V>::T;
     const int d = (int)p.pd.d;
     const int R = p.R;
     const int tid = threadIdx.x;
-    const int d8 = d / 8;
-    float* data = (float*)smem;
+    VT* tile = (VT*)smem;
     unsigned char* stage_buf = smem + (size_t)R * d * sizeof(float);
     uint64_t* bar = (uint64_t*)(stage_buf + (p.staged ? (size_t)R * d * sizeof(TIn) : 0));
 
-    int64_t tile = blockIdx.x;
-    if (tile >= p.ntiles) return;
+    int64_t t_idx = blockIdx.x;
+    if (t_idx >= p.ntiles) return;
     if (p.staged) {
         if (tid == 0) mbar_init(bar, 1);
         __syncthreads();
-        if (tid == 0) issue_tile<TIn>(p, tile, stage_buf, bar);
+        if (tid == 0) issue_tile<TIn>(p, t_idx, stage_buf, bar);
     }
     uint32_t parity = 0;
-    for (; tile < p.ntiles; tile += gridDim.x) {
-        const int64_t row0 = tile * R;
+    for (; t_idx < p.ntiles; t_idx += gridDim.x) {
+        const int64_t row0 = t_idx * R;
         const int nr = (int)min((int64_t)R, p.rows - row0);
-        // rows -> fp32 tile
+        const int qv = (nr + V - 1) / V;
         if (p.staged) {
             const bool ok = mbar_wait(bar, parity);
             parity ^= 1;
@@ -278,34 +350,22 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
                 if (tid == 0) atomicExch(p.status, 1);
                 return;
             }
-            const TIn* src = (const TIn*)stage_buf;
-            for (int r = 0; r < nr; ++r)
-                for (int j = tid; j < d8; j += kThreads) {
-                    float v[8];
-                    load8(src + (size_t)r * d + 8 * j, v);
-                    store8(data + r * d + swz(8 * j, p.swz), v);
-                }
+            fill_tile<V, TIn>(tile, d, nr, (const TIn*)stage_buf, d, p.mask);
         } else {
-            const TIn* x = (const TIn*)p.x;
-            for (int r = 0; r < nr; ++r)
-                for (int j = tid; j < d8; j += kThreads) {
-                    float v[8];
-                    load8(x + (row0 + r) * p.ld_x + 8 * j, v);
-                    store8(data + r * d + swz(8 * j, p.swz), v);
-                }
+            fill_tile<V, TIn>(tile, d, nr, (const TIn*)p.x + row0 * p.ld_x, p.ld_x, p.mask);
         }
         __syncthreads();
-        if (p.staged && tid == 0 && tile + gridDim.x < p.ntiles) {
+        if (p.staged && tid == 0 && t_idx + gridDim.x < p.ntiles) {
             fence_proxy_async_smem();   // the staging reads above happen before the copies' writes
-            issue_tile<TIn>(p, tile + gridDim.x, stage_buf, bar);
+            issue_tile<TIn>(p, t_idx + gridDim.x, stage_buf, bar);
         }
         for (int step = 0; step < p.pd.m; ++step) {
             const int t = INV ? p.pd.m - 1 - step : step;
             const StageDesc& sd = p.pd.st[t];
             switch (sd.b) {
-#define HARP_TILED_CASE(R)                                                         \
-    case R:                                                                        \
-        if constexpr ((MASK >> R) & 1) run_stage<R, INV>(sd, p.blocks, data, d, nr, p.swz); \
+#define HARP_TILED_CASE(R)                                                     \
+    case R:                                                                    \
+        if constexpr ((MASK >> R) & 1) run_stage<R, INV, V>(sd, p.lanes + p.lane_off[t], tile, d, qv, p.mask); \
         break;
                 HARP_TILED_CASE(2) HARP_TILED_CASE(3) HARP_TILED_CASE(4) HARP_TILED_CASE(5)
                 HARP_TILED_CASE(6) HARP_TILED_CASE(7) HARP_TILED_CASE(8)
@@ -314,13 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
             }
             __syncthreads();
         }
-        TOut* y = (TOut*)p.y;
-        for (int r = 0; r < nr; ++r)
-            for (int j = tid; j < d8; j += kThreads) {
-                float v[8];
-                load8(data + r * d + swz(8 * j, p.swz), v);
-                store8(y + (row0 + r) * p.ld_y + 8 * j, v);
-            }
+        drain_tile<V, TOut>(tile, d, nr, (TOut*)p.y + row0 * p.ld_y, p.ld_y, p.mask);
         __syncthreads();
     }
 }
@@ -332,32 +386,44 @@ constexpr int kMasks[] = {1 << 8, (1 << 2) | (1 << 8), (1 << 2) | (1 << 5) | (1 
                           (1 << 2) | (1 << 7) | (1 << 8), 0x1fc};
 constexpr int kNumMasks = sizeof(kMasks) / sizeof(kMasks[0]);
 
-template <typename TIn, typename TOut, bool INV, int I>
+// Sub-tiles of one row (V = 1) are needed only when four fp32 rows do not fit in shared
+// memory (d > 14524); they are built for the radix sets without 5.
+constexpr bool has_row_major_kernel(int mask) { return ((mask >> 5) & 1) == 0; }
+
+template <typename TIn, typename TOut, bool INV, int V, int I>
 cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
     if constexpr (I < kNumMasks) {
-        if (which != I) return launch_mask<TIn, TOut, INV, I + 1>(which, tp, smem, grid, stream);
-        auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I]>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<(unsigned)grid, kThreads, smem, stream>>>(tp);
-        return cudaGetLastError();
+        if (which != I) return launch_mask<TIn, TOut, INV, V, I + 1>(which, tp, smem, grid, stream);
+        if constexpr (V == 1 && !has_row_major_kernel(kMasks[I])) {
+            return cudaErrorInvalidValue;
+        } else {
+            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<(unsigned)grid, kThreads, smem, stream>>>(tp);
+            return cudaGetLastError();
+        }
     } else {
         return cudaErrorInvalidValue;
     }
 }
 
 template <typename TIn, typename TOut>
-cudaError_t launch(int which, bool inverse, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
-    return inverse ? launch_mask<TIn, TOut, true, 0>(which, tp, smem, grid, stream)
-                   : launch_mask<TIn, TOut, false, 0>(which, tp, smem, grid, stream);
+cudaError_t launch(int which, int V, bool inverse, const TiledParams& tp, size_t smem, int grid,
+                   cudaStream_t stream) {
+    if (V == 4)
+        return inverse ? launch_mask<TIn, TOut, true, 4, 0>(which, tp, smem, grid, stream)
+                       : launch_mask<TIn, TOut, false, 4, 0>(which, tp, smem, grid, stream);
+    return inverse ? launch_mask<TIn, TOut, true, 1, 0>(which, tp, smem, grid, stream)
+                   : launch_mask<TIn, TOut, false, 1, 0>(which, tp, smem, grid, stream);
 }
 
 }  // namespace harp_tiled
 
 // One translation unit per I/O type pair (compiled in parallel).
-cudaError_t harp_tiled_launch_bf16(int which, bool inverse, const harp_tiled::TiledParams& tp, size_t smem,
-                                   int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_f32(int which, bool inverse, const harp_tiled::TiledParams& tp, size_t smem,
-                                  int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_bf16_f32(int which, bool inverse, const harp_tiled::TiledParams& tp, size_t smem,
-                                       int grid, cudaStream_t stream);
+cudaError_t harp_tiled_launch_bf16(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+                                   size_t smem, int grid, cudaStream_t stream);
+cudaError_t harp_tiled_launch_f32(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+                                  size_t smem, int grid, cudaStream_t stream);
+cudaError_t harp_tiled_launch_bf16_f32(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+                                       size_t smem, int grid, cudaStream_t stream);

@@ -36,11 +36,19 @@ struct harp_plan_s {
     std::map<int, int> mixer_index;             // radix -> offset into mixers
     int64_t theta_total = 0;
     int64_t block_floats = 0;
+    // Lane-interleaved copy of the blocks for the tiled kernel: per stage, blocks in groups
+    // of 32 consecutive c; inside a group, 16-byte piece q of block c at
+    // (group * (b*b/4) + q) * 32 + (c % 32) (in float4 units) when b*b % 4 == 0, else
+    // float e of block c at (group * b*b + e) * 32 + (c % 32).  A warp whose lanes take 32
+    // consecutive blocks then reads 512 (128) contiguous bytes per load.
+    int64_t lane_off[HARP_MAX_STAGES] = {0};
+    int64_t lane_floats = 0;
 
     // device side (owned)
     int device = -1;
     bool materialized = false;
     float* d_blocks = nullptr;        // signed blocks, [stage][c][k][l]
+    float* d_blocks_lanes = nullptr;  // the same, lane-interleaved (see lane_off)
     void* d_theta = nullptr;          // float or int8 codes, as stored
     float* d_scales = nullptr;
     double* d_mixers = nullptr;

@@ -86,6 +86,19 @@ __global__ void materialize_kernel(PlanDesc pd, const float* __restrict__ theta_
     }
 }
 
+// Blocks of one stage -> the lane-interleaved layout described in harp_internal.h.
+__global__ void interleave_kernel(const float* __restrict__ src, float* __restrict__ dst, int64_t nb, int bb) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= nb * bb) return;
+    const int64_t c = idx / bb;
+    const int e = (int)(idx - c * bb);
+    const int64_t group = c >> 5, lane = c & 31;
+    int64_t to;
+    if (bb % 4 == 0) to = ((group * (bb / 4) + e / 4) * 32 + lane) * 4 + (e & 3);
+    else to = (group * bb + e) * 32 + lane;
+    dst[to] = src[idx];
+}
+
 template <typename T>
 harp_status dev_alloc_copy(T** dst, const T* src, size_t n, cudaStream_t stream) {
     if (*dst == nullptr) {
@@ -109,12 +122,13 @@ harp_status harp_device_free(harp_plan_s* p) {
     cudaDeviceSynchronize();
     fast_state_free(p);
     cudaFree(p->d_blocks);
+    cudaFree(p->d_blocks_lanes);
     cudaFree(p->d_theta);
     cudaFree(p->d_scales);
     cudaFree(p->d_mixers);
     cudaFree(p->d_signs);
     cudaFree(p->d_status);
-    p->d_blocks = nullptr; p->d_theta = nullptr; p->d_scales = nullptr;
+    p->d_blocks = nullptr; p->d_blocks_lanes = nullptr; p->d_theta = nullptr; p->d_scales = nullptr;
     p->d_mixers = nullptr; p->d_signs = nullptr; p->d_status = nullptr;
     p->materialized = false;
     p->device = -1;
@@ -153,6 +167,13 @@ extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream_) {
         cudaGetLastError();
         return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the blocks failed");
     }
+    if (!p->d_blocks_lanes) {
+        if (cudaMalloc((void**)&p->d_blocks_lanes, sizeof(float) * p->lane_floats) != cudaSuccess) {
+            cudaGetLastError();
+            return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the interleaved blocks failed");
+        }
+        cudaMemsetAsync(p->d_blocks_lanes, 0, sizeof(float) * p->lane_floats, stream);
+    }
     if (!p->d_status) {
         if (cudaMalloc((void**)&p->d_status, 64) != cudaSuccess) {
             cudaGetLastError();
@@ -169,6 +190,12 @@ extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream_) {
         p->desc, p->kind == HARP_THETA_F32 ? (const float*)p->d_theta : nullptr,
         p->kind == HARP_THETA_I8 ? (const int8_t*)p->d_theta : nullptr, p->d_scales, p->d_mixers,
         p->d_signs, p->d_blocks, total);
+    for (int t = 0; t < p->desc.m; ++t) {
+        const StageDesc& sd = p->desc.st[t];
+        const int64_t n = sd.nblocks * sd.b * sd.b;
+        interleave_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+            p->d_blocks + sd.block_off, p->d_blocks_lanes + p->lane_off[t], sd.nblocks, sd.b * sd.b);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     p->materialized = true;

@@ -178,7 +178,7 @@ harp_status harp_plan_create(harp_plan_t* out, int64_t d, const int32_t* radices
         p->kind = kind;
         p->sign_seed = sign_seed;
         p->qr_seed = qr_seed;
-        int64_t s = 1, toff = 0, boff = 0;
+        int64_t s = 1, toff = 0, boff = 0, loff = 0;
         for (int t = 0; t < m; ++t) {
             StageDesc& sd = p->desc.st[t];
             sd.b = radices[t];
@@ -187,12 +187,15 @@ harp_status harp_plan_create(harp_plan_t* out, int64_t d, const int32_t* radices
             sd.nblocks = d / sd.b;
             sd.theta_off = toff;
             sd.block_off = boff;
+            p->lane_off[t] = loff;
             s *= sd.b;
             toff += sd.nblocks * sd.p;
             boff += sd.nblocks * sd.b * sd.b;
+            loff += (sd.nblocks + 31) / 32 * 32 * sd.b * sd.b;
         }
         p->theta_total = toff;
         p->block_floats = boff;
+        p->lane_floats = loff;
 
         if (kind == HARP_THETA_F32) {
             p->theta_f32.assign(toff, 0.0f);
