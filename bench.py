@@ -27,6 +27,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from structured_rotations_b200.shard import max_over_ranks, weak_shard  # noqa: E402
+
 METRIC = "HARP rotation rows/s and HBM GB/s (fraction of B200 roofline), d=4096/5120/8192"
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -71,6 +73,11 @@ def peaks():
 # ----------------------------------------------------------------- clocks ---
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled during the timed region: NVML polled
+    every 5 ms from a thread, or `nvidia-smi -lms 100` when NVML is not importable.
+    Read-only queries; no GPU setting is touched."""
+    REASONS = ((0x8, "hw_slowdown"), (0x40, "hw_thermal_slowdown"), (0x20, "sw_thermal_slowdown"),
+               (0x4, "sw_power_cap"), (0x80, "hw_power_brake_slowdown"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -79,8 +86,43 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.samples = []
+        self.stop_flag = False
+        self.nvml = None
+        self.handle = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        try:
+            self.nvml, self.handle = self._nvml_handle()
+            self.max_mhz = self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+            import threading
+
+            def loop():
+                while not self.stop_flag:
+                    try:
+                        sm = self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM)
+                        rs = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                        self.samples.append((sm, rs))
+                    except Exception:
+                        pass
+                    time.sleep(0.005)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.nvml = None
         fd, self.path = tempfile.mkstemp(prefix="harp_clocks_", suffix=".csv")
         os.close(fd)
         try:
@@ -92,6 +134,18 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+            reasons = set()
+            for _, rs in self.samples:
+                for bit, name in self.REASONS:
+                    if rs & bit:
+                        reasons.add(name)
+            return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml, 5 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -112,7 +166,7 @@ class ClockSampler:
                     continue
         os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "nvidia-smi"}
         load = [r for r in rows if r["util"] >= 50] or rows
         reasons = set()
         for r in load:
@@ -121,7 +175,7 @@ class ClockSampler:
                 if r[key].lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["max"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(load)}
+                "reasons": sorted(reasons), "samples": len(load), "source": "nvidia-smi, 100 ms"}
 
 
 # --------------------------------------------------------------- profiles ---
@@ -277,10 +331,7 @@ def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        tm = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tm.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e = {"value": world * rows * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
            "path": "pinned host -> device copy, harp_apply, device -> pinned host copy, one stream"}
@@ -313,7 +364,8 @@ def run_ours(args):
     rows, d = w.rows, w.d
     plan = make_plan(args.workload, H, W)
     t = time.time()
-    enc = W.draw_encoded(w, rank * rows, rows)       # this rank's shard of the global batch
+    row0, rows = weak_shard(rows, rank)              # this rank's block of the global batch
+    enc = W.draw_encoded(w, row0, rows)
     log(f"rank {rank}: generated {rows}x{d} input in {time.time() - t:.1f}s")
     x = to_device_bf16(enc, torch, device)
     y = torch.empty_like(x)
@@ -323,10 +375,7 @@ def run_ours(args):
     elapsed, kern_ms, launches, kname = time_apply(plan, x, y, args.steps, args.warmup, torch, dist)
     clocks = sampler.stop()
 
-    if dist is not None:
-        tm = torch.tensor([elapsed], device=device, dtype=torch.float64)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        elapsed = float(tm.item())
+    elapsed = max_over_ranks(elapsed, dist, device)
     step_ms = elapsed / args.steps
     value = world * rows * args.steps / (elapsed / 1e3)
     bytes_per_launch = 2 * rows * d * 2

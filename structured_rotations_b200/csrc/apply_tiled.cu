@@ -49,30 +49,26 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     while (which < kNumMasks && (kMasks[which] & mask) != mask) ++which;
     if (which == kNumMasks) return HARP_ERR_UNSUPPORTED;
 
-    // Rows per tile R = V Q: Q sub-tiles of V = 4 rows (fp32, 16 d bytes each), plus a
-    // staging area for the next tile's raw rows unless staging would halve Q; sub-tiles of
-    // one row when not even one 4-row sub-tile fits.
+    // Rows per tile R = V Q: as many sub-tiles of V = 4 rows (fp32, 16 d bytes each) as fit,
+    // then as many of the next tile's raw rows as fit in the rest go to a staging area
+    // (bulk copies overlap the arithmetic; the other rows are read directly).  One
+    // sub-tile fewer when that would stage fewer than half the rows.  Sub-tiles of one
+    // row when not even one 4-row sub-tile fits.
     const int64_t budget = kSmemOptIn - 64;
-    const int64_t q_staged = std::min<int64_t>(budget / (4 * d * (4 + es_in)), kMaxTileRows / 4);
-    const int64_t q_plain = std::min<int64_t>(budget / (16 * d), kMaxTileRows / 4);
-    int V = 4, staged = 1;
-    int64_t Q = q_staged;
-    if (q_plain >= 2 * q_staged) {
-        Q = q_plain;
-        staged = 0;
-    }
+    auto staged_for = [&](int64_t r) {
+        return std::max<int64_t>(0, std::min<int64_t>(r, (budget - r * d * 4) / (d * es_in)));
+    };
+    int V = 4;
+    int64_t Q = std::min<int64_t>(budget / (16 * d), kMaxTileRows / 4);
+    if (Q > 1 && staged_for(4 * Q) < 2 * Q) --Q;
     if (Q < 1) {
         V = 1;
-        Q = std::min<int64_t>(budget / (d * (4 + es_in)), kMaxTileRows);
-        staged = 1;
-        if (Q < 2) {
-            Q = std::min<int64_t>(budget / (d * 4), kMaxTileRows);
-            staged = 0;
-        }
+        Q = std::min<int64_t>(budget / (4 * d), kMaxTileRows);
         if (Q < 1 || !has_row_major_kernel(kMasks[which])) return HARP_ERR_UNSUPPORTED;
     }
     Q = std::min<int64_t>(Q, (rows + V - 1) / V);
     const int64_t R = V * Q;
+    const int64_t staged = std::min<int64_t>(staged_for(R), rows);
 
     TiledParams tp;
     tp.pd = p->desc;
@@ -85,10 +81,10 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.ld_y = ld_y;
     tp.ntiles = (rows + R - 1) / R;
     tp.R = (int)R;
-    tp.staged = staged;
+    tp.staged_rows = (int)staged;
     tp.mask = (d % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
-    const size_t smem = (size_t)R * d * 4 + (staged ? (size_t)R * d * es_in : 0) + 16;
+    const size_t smem = (size_t)R * d * 4 + (size_t)staged * d * es_in + 16;
     const int grid = (int)std::min<int64_t>(tp.ntiles, sm_count());
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;

@@ -49,7 +49,7 @@ struct TiledParams {
     int64_t rows, ld_x, ld_y;   // in elements
     int64_t ntiles;
     int R;                      // rows per tile (a multiple of the sub-tile height V)
-    int staged;                 // 1: rows of the next tile arrive by bulk copy
+    int staged_rows;            // the first rows of the next tile that arrive by bulk copy
     int mask;                   // V = 1 swizzle: 0x18 when d % 32 == 0, else 0
     int* status;
 };
@@ -143,9 +143,10 @@ __device__ __forceinline__ void store8(__nv_bfloat16* dst, const float (&v)[8]) 
 }
 
 // Block B_{t,c} (b*b floats, row-major [output k][input l]) from the stage's
-// lane-interleaved copy: lanes holding 32 consecutive c read contiguous memory.
+// lane-interleaved copy: lanes holding 32 consecutive c read contiguous memory.  The
+// buffer holds the largest block (8 x 8); a radix-b stage uses its first b*b entries.
 template <int B>
-__device__ __forceinline__ void load_block(float (&w)[B * B], const float* __restrict__ stage, int c) {
+__device__ __forceinline__ void load_block(float (&w)[64], const float* __restrict__ stage, int c) {
     const int group = c >> 5, lane = c & 31;
     if constexpr ((B * B) % 4 == 0) {
         const float4* src = (const float4*)stage + (size_t)group * (B * B / 4) * 32 + lane;
@@ -158,6 +159,26 @@ __device__ __forceinline__ void load_block(float (&w)[B * B], const float* __res
         const float* src = stage + (size_t)group * (B * B) * 32 + lane;
 #pragma unroll
         for (int e = 0; e < B * B; ++e) w[e] = __ldg(src + e * 32);
+    }
+}
+
+// The same for a radix known only at run time (the first block of the next stage).
+__device__ __forceinline__ void load_block_any(float (&w)[64], const float* __restrict__ stage, int c, int bb) {
+    const int group = c >> 5, lane = c & 31;
+    if ((bb & 3) == 0) {
+        const float4* src = (const float4*)stage + (size_t)group * (bb / 4) * 32 + lane;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (4 * q < bb) {
+                const float4 v = __ldg(src + q * 32);
+                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+            }
+        }
+    } else {
+        const float* src = stage + (size_t)group * bb * 32 + lane;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+            if (e < bb) w[e] = __ldg(src + e * 32);
     }
 }
 
@@ -174,44 +195,42 @@ __device__ __forceinline__ void zero_v(float& v) { v = 0.f; }
 // One group in one sub-tile (V rows at once): y = B x (forward) or B^T x (inverse), in
 // place.  Each output is summed as fma(B[k][l], x_l, acc) over l = 0..b-1 from zero.
 template <int B, bool INV, typename VT>
-__device__ __forceinline__ void group_vec(VT* __restrict__ st, const int (&pos)[B], const float (&w)[B * B]) {
+__device__ __forceinline__ void group_vec(VT* __restrict__ st, const int (&pos)[B], const float (&w)[64]) {
     VT xv[B];
 #pragma unroll
     for (int l = 0; l < B; ++l) xv[l] = st[pos[l]];
+    // l outer, k inner: consecutive FMAs update different outputs, so dependent FMAs are
+    // 4 B instructions apart; every output still sums over l = 0..b-1 in order.
     VT yv[B];
 #pragma unroll
-    for (int k = 0; k < B; ++k) {
-        zero_v(yv[k]);
+    for (int k = 0; k < B; ++k) zero_v(yv[k]);
 #pragma unroll
-        for (int l = 0; l < B; ++l) fma_v(yv[k], INV ? w[l * B + k] : w[k * B + l], xv[l]);
-    }
+    for (int l = 0; l < B; ++l)
+#pragma unroll
+        for (int k = 0; k < B; ++k) fma_v(yv[k], INV ? w[l * B + k] : w[k * B + l], xv[l]);
 #pragma unroll
     for (int k = 0; k < B; ++k) st[pos[k]] = yv[k];
 }
 
-// Item = (block c, sub-tile group g): the sub-tiles g, g + G, ... of the tile.
+// Item = (block c, sub-tile group g): the sub-tiles g, g + G, ... of the tile; block c
+// has lo = c % s, hi = c / s.  The caller steps (c, g, lo, hi) from item to item.
+struct ItemPos {
+    int c, g, lo, hi;
+};
+
 template <int B, bool INV, int V>
-__device__ __forceinline__ void apply_item(typename VecOf<V>::T* tile, int d, int qv, int G, int nb, int s,
-                                           int mask, int item, const float (&w)[B * B]) {
-    const int c = item % nb;
-    const int g = item / nb;
-    const int lo = c % s, hi = c / s;
-    const int base = lo + s * B * hi;
+__device__ __forceinline__ void apply_item(typename VecOf<V>::T* tile, int d, int qv, int G, int s, int mask,
+                                           const ItemPos& it, const float (&w)[64]) {
+    const int base = it.lo + s * B * it.hi;
     int pos[B];
 #pragma unroll
     for (int k = 0; k < B; ++k) pos[k] = slot<V>(base + s * k, mask);
-    for (int q = g; q < qv; q += G) group_vec<B, INV>(tile + q * d, pos, w);
+    for (int q = it.g; q < qv; q += G) group_vec<B, INV>(tile + q * d, pos, w);
 }
 
-// All items of one stage; the coefficients of the thread's next item are loaded while
-// the current one is applied.
-template <int B, bool INV, int V>
-__device__ __forceinline__ void run_stage(const StageDesc& sd, const float* __restrict__ sb,
-                                          typename VecOf<V>::T* tile, int d, int qv, int mask) {
-    const int nb = d / B;
-    const int s = (int)sd.s;
-    // Sub-tile groups: split the tile's sub-tiles over more items only while too few
-    // items would leave a fifth or more of the threads' slots empty.
+// Sub-tile groups of a stage: split the tile's sub-tiles over more items only while
+// too few items would leave a fifth or more of the threads' slots empty.
+__device__ __forceinline__ int stage_groups(int nb, int qv) {
     int G = 1;
     while (G < qv) {
         const int items = nb * G;
@@ -219,22 +238,77 @@ __device__ __forceinline__ void run_stage(const StageDesc& sd, const float* __re
         if (per * kThreads * 4 <= items * 5) break;
         ++G;
     }
+    return G;
+}
+
+// What a thread prefetches after its last item of a stage: the first block it will
+// apply in the next stage (of this tile, or stage 0 of its next tile).
+struct NextFirst {
+    const float* stage;   // lane-interleaved blocks of that stage (nullptr: nothing)
+    int nb, bb;
+};
+
+// All items of one stage.  Coefficients are double-buffered in wa / wb: on entry the
+// buffer named by cur_a holds (or is loading) the thread's first block of this stage;
+// while an item is applied the other buffer loads the next one, which after the last
+// item is the first block of the next stage, so on exit cur_a names that buffer.
+template <int B, bool INV, int V>
+__device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, typename VecOf<V>::T* tile,
+                                          int d, int qv, int mask, float (&wa)[64], float (&wb)[64],
+                                          bool& cur_a, const NextFirst& nx) {
+    const int nb = d / B;
+    const int G = stage_groups(nb, qv);
     const int items = nb * G;
-    int j = threadIdx.x;
-    if (j >= items) return;
-    float wa[B * B], wb[B * B];
-    load_block<B>(wa, sb, j % nb);
+    const int tid = threadIdx.x;
+    int j = tid;
+    if (j >= items) {   // idle in this stage: start loading the next stage's block now
+        if (nx.stage) {
+            if (cur_a) load_block_any(wa, nx.stage, tid % nx.nb, nx.bb);
+            else load_block_any(wb, nx.stage, tid % nx.nb, nx.bb);
+        }
+        return;
+    }
+    // Items j = tid, tid + T, ...: c = j % nb, g = j / nb, and for the block lo = c % s,
+    // hi = c / s, stepped by T without dividing (T % s, T / s once per stage).
+    ItemPos it;
+    it.c = tid % nb;
+    it.g = tid / nb;
+    it.lo = it.c % s;
+    it.hi = it.c / s;
+    const int dlo = kThreads % s, dhi = kThreads / s;
     while (true) {
-        int jn = j + kThreads;
-        if (jn < items) load_block<B>(wb, sb, jn % nb);
-        apply_item<B, INV, V>(tile, d, qv, G, nb, s, mask, j, wa);
+        const int jn = j + kThreads;
+        ItemPos nt = it;
+        nt.c += kThreads;
+        nt.lo += dlo;
+        nt.hi += dhi;
+        if (nt.lo >= s) {
+            nt.lo -= s;
+            ++nt.hi;
+        }
+        if (nt.c >= nb) {   // wrapped into the next sub-tile group (small nb only)
+            nt.c -= nb;
+            ++nt.g;
+            while (nt.c >= nb) {
+                nt.c -= nb;
+                ++nt.g;
+            }
+            nt.lo = nt.c % s;
+            nt.hi = nt.c / s;
+        }
+        if (cur_a) {
+            if (jn < items) load_block<B>(wb, sb, nt.c);
+            else if (nx.stage) load_block_any(wb, nx.stage, tid % nx.nb, nx.bb);
+            apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, wa);
+        } else {
+            if (jn < items) load_block<B>(wa, sb, nt.c);
+            else if (nx.stage) load_block_any(wa, nx.stage, tid % nx.nb, nx.bb);
+            apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, wb);
+        }
+        cur_a = !cur_a;
         if (jn >= items) break;
         j = jn;
-        jn = j + kThreads;
-        if (jn < items) load_block<B>(wa, sb, jn % nb);
-        apply_item<B, INV, V>(tile, d, qv, G, nb, s, mask, j, wb);
-        if (jn >= items) break;
-        j = jn;
+        it = nt;
     }
 }
 
@@ -243,7 +317,7 @@ __device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, u
                                            uint64_t* bar) {
     const int d = (int)p.pd.d;
     const int64_t row0 = tile * p.R;
-    const int nr = (int)min((int64_t)p.R, p.rows - row0);
+    const int nr = (int)min((int64_t)p.staged_rows, p.rows - row0);
     const uint32_t row_bytes = (uint32_t)d * sizeof(TIn);
     mbar_arrive_expect_tx(bar, row_bytes * nr);
     const TIn* x = (const TIn*)p.x;
@@ -255,9 +329,11 @@ __device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, u
 // 16-byte stores (the XOR keeps 8-aligned runs contiguous).  Rows past the end of the
 // batch are zero.
 template <int V, typename TIn>
-__device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int nr, const TIn* src, int64_t ld,
-                                          int mask) {
+__device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int nr, int n_staged, const TIn* staged,
+                                          const TIn* src, int64_t ld, int mask) {
     const int d8 = d / 8;
+    // row r of the tile: the staging area for r < n_staged, else global memory
+    auto row_ptr = [&](int r) -> const TIn* { return r < n_staged ? staged + (size_t)r * d : src + r * ld; };
     for (int q = 0; V * q < nr; ++q)
         for (int j = threadIdx.x; j < d8; j += kThreads) {
             if constexpr (V == 4) {
@@ -265,7 +341,7 @@ __device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if (4 * q + e < nr) {
-                        load8(src + (4 * q + e) * ld + 8 * j, v[e]);
+                        load8(row_ptr(4 * q + e) + 8 * j, v[e]);
                     } else {
 #pragma unroll
                         for (int k = 0; k < 8; ++k) v[e][k] = 0.0f;
@@ -276,7 +352,7 @@ __device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int
                 for (int k = 0; k < 8; ++k) st[slot<4>(8 * j + k, mask)] = make_float4(v[0][k], v[1][k], v[2][k], v[3][k]);
             } else {
                 float v[8];
-                load8(src + q * ld + 8 * j, v);
+                load8(row_ptr(q) + 8 * j, v);
                 store8(tile + q * d + slot<1>(8 * j, mask), v);
             }
         }
@@ -325,47 +401,74 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
     extern __shared__ __align__(128) unsigned char smem[];
     using VT = typename VecOf<V>::T;
     const int d = (int)p.pd.d;
+    const int m = p.pd.m;
     const int R = p.R;
     const int tid = threadIdx.x;
     VT* tile = (VT*)smem;
     unsigned char* stage_buf = smem + (size_t)R * d * sizeof(float);
-    uint64_t* bar = (uint64_t*)(stage_buf + (p.staged ? (size_t)R * d * sizeof(TIn) : 0));
+    uint64_t* bar = (uint64_t*)(stage_buf + (size_t)p.staged_rows * d * sizeof(TIn));
 
     int64_t t_idx = blockIdx.x;
     if (t_idx >= p.ntiles) return;
-    if (p.staged) {
+    if (p.staged_rows) {
         if (tid == 0) mbar_init(bar, 1);
         __syncthreads();
         if (tid == 0) issue_tile<TIn>(p, t_idx, stage_buf, bar);
+    }
+    // The stage order: forward 0..m-1, inverse m-1..0.
+    auto stage_of = [&](int step) { return INV ? m - 1 - step : step; };
+    auto first_of = [&](int step, int qv_) {
+        const int t = stage_of(step);
+        const int b = p.pd.st[t].b, nb = d / b;
+        NextFirst f;
+        f.stage = tid < nb * stage_groups(nb, qv_) ? p.lanes + p.lane_off[t] : nullptr;
+        f.nb = nb;
+        f.bb = b * b;
+        return f;
+    };
+    float wa[64], wb[64];
+    bool cur_a = true;
+    {
+        const int nr0 = (int)min((int64_t)R, p.rows - t_idx * R);
+        const NextFirst f = first_of(0, (nr0 + V - 1) / V);
+        if (f.stage) load_block_any(wa, f.stage, tid % f.nb, f.bb);
     }
     uint32_t parity = 0;
     for (; t_idx < p.ntiles; t_idx += gridDim.x) {
         const int64_t row0 = t_idx * R;
         const int nr = (int)min((int64_t)R, p.rows - row0);
         const int qv = (nr + V - 1) / V;
-        if (p.staged) {
+        const int n_staged = min(nr, p.staged_rows);
+        if (n_staged) {
             const bool ok = mbar_wait(bar, parity);
             parity ^= 1;
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) atomicExch(p.status, 1);
                 return;
             }
-            fill_tile<V, TIn>(tile, d, nr, (const TIn*)stage_buf, d, p.mask);
-        } else {
-            fill_tile<V, TIn>(tile, d, nr, (const TIn*)p.x + row0 * p.ld_x, p.ld_x, p.mask);
         }
+        fill_tile<V, TIn>(tile, d, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x, p.ld_x,
+                          p.mask);
         __syncthreads();
-        if (p.staged && tid == 0 && t_idx + gridDim.x < p.ntiles) {
+        const int64_t t_next = t_idx + gridDim.x;
+        if (p.staged_rows && tid == 0 && t_next < p.ntiles) {
             fence_proxy_async_smem();   // the staging reads above happen before the copies' writes
-            issue_tile<TIn>(p, t_idx + gridDim.x, stage_buf, bar);
+            issue_tile<TIn>(p, t_next, stage_buf, bar);
         }
-        for (int step = 0; step < p.pd.m; ++step) {
-            const int t = INV ? p.pd.m - 1 - step : step;
+        const int nr_next = t_next < p.ntiles ? (int)min((int64_t)R, p.rows - t_next * R) : 0;
+        for (int step = 0; step < m; ++step) {
+            const int t = stage_of(step);
             const StageDesc& sd = p.pd.st[t];
+            NextFirst nx;
+            if (step + 1 < m) nx = first_of(step + 1, qv);
+            else if (nr_next) nx = first_of(0, (nr_next + V - 1) / V);
+            else nx.stage = nullptr, nx.nb = 1, nx.bb = 0;
+            const float* sb = p.lanes + p.lane_off[t];
+            const int s = (int)sd.s;
             switch (sd.b) {
-#define HARP_TILED_CASE(R)                                                     \
-    case R:                                                                    \
-        if constexpr ((MASK >> R) & 1) run_stage<R, INV, V>(sd, p.lanes + p.lane_off[t], tile, d, qv, p.mask); \
+#define HARP_TILED_CASE(R)                                                                       \
+    case R:                                                                                      \
+        if constexpr ((MASK >> R) & 1) run_stage<R, INV, V>(sb, s, tile, d, qv, p.mask, wa, wb, cur_a, nx); \
         break;
                 HARP_TILED_CASE(2) HARP_TILED_CASE(3) HARP_TILED_CASE(4) HARP_TILED_CASE(5)
                 HARP_TILED_CASE(6) HARP_TILED_CASE(7) HARP_TILED_CASE(8)
