@@ -36,6 +36,8 @@ WORKLOAD_TEXT = {
     "c2": "d=4096 schedule (8,8,8,8), 65536 rows/GPU bf16 Student-t(3) with 8 outlier channels x50, "
           "theta~N(0,0.05), forward",
     "c3_64k": "d=5120 schedule (8,8,8,5,2), 65536 rows/GPU bf16 N(0,1) with 1% entries x20, forward",
+    "c4": "two-sided T_U^T W T_V: W 28672x8192 bf16 N(0,0.02^2) with 16 outlier columns x30, "
+          "U (8,8,8,8,7), V (8,8,8,8,2), theta~N(0,0.05)",
     "c5": "d=8192 schedule (8,8,8,8,2), int8 theta + per-stage scale, 65536 rows/GPU bf16 N(0,1), forward",
 }
 
@@ -50,7 +52,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3_64k", "c5"])
     ap.add_argument("--no-extra", action="store_true", help="skip the d=5120 / d=8192 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -284,13 +286,13 @@ def cpu_baseline(args, W):
 
 # ------------------------------------------------------------------ ours ---
 
-def time_apply(plan, x, y, steps, warmup, torch, dist=None):
+def time_apply(plan, x, y, steps, warmup, torch, dist=None, direction="forward"):
     """Warm up, then time exactly `steps` applies between a barrier and a sync on
     both sides.  Returns (elapsed_ms, mean kernel ms, launches)."""
     import structured_rotations_b200 as H
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
-        plan.apply(x, y)
+        plan.apply(x, y, direction=direction)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -301,7 +303,7 @@ def time_apply(plan, x, y, steps, warmup, torch, dist=None):
     t0.record(stream)
     for a, b in ev:
         a.record(stream)
-        plan.apply(x, y)
+        plan.apply(x, y, direction=direction)
         b.record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -337,6 +339,60 @@ def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
            "path": "pinned host -> device copy, harp_apply, device -> pinned host copy, one stream"}
     del xh, yh
     return e2e
+
+
+SIDE = (("c2", "inverse"), ("c3_64k", "forward"), ("c3_64k", "inverse"), ("c5", "forward"),
+        ("c5", "inverse"))
+
+
+def side_measurements(args, H, W, torch, device, peak):
+    """The other configurations' rows/s and GB/s (device-timed, one line each): every
+    direction the workloads list, and the two-sided weight rotation."""
+    out = []
+    cache = {}
+    for name, direction in SIDE:
+        ww = W.get(name)
+        if name not in cache:
+            cache.clear()
+            e2 = W.draw_encoded(ww, 0, ww.rows)
+            cache[name] = (make_plan(name, H, W), to_device_bf16(e2, torch, device))
+        p2, x2 = cache[name]
+        y2 = torch.empty_like(x2)
+        st = max(3, args.steps // 4)
+        el, km, _, kn = time_apply(p2, x2, y2, st, max(3, args.warmup // 2), torch, direction=direction)
+        b2 = 2 * ww.rows * ww.d * 2
+        out.append({"workload": WORKLOAD_TEXT[name].replace("forward", direction), "rows_per_s": ww.rows * st / (el / 1e3),
+                    "hbm_gbs": b2 / (km / 1e3) / 1e9, "hbm_frac": b2 / (km / 1e3) / 1e9 / peak,
+                    "kernel": kn, "kernel_ms": km,
+                    "traffic": recorded_traffic(kn, name) if direction == "forward" else None})
+        del y2
+    cache.clear()
+    # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)
+    w4 = W.get("c4")
+    th_v = W.draw_theta(H.theta_count(w4.schedule), w4.theta_sigma, w4.theta_seed)
+    th_u = W.draw_theta(H.theta_count(w4.u_schedule), w4.theta_sigma, w4.theta_seed + 7)
+    pv = H.Plan(w4.n_in, w4.schedule, theta=th_v, sign_seed=w4.sign_seed).materialize()
+    pu = H.Plan(w4.n_out, w4.u_schedule, theta=th_u, sign_seed=w4.sign_seed + 11).materialize()
+    wt = to_device_bf16(W.draw_encoded(w4, 0, w4.n_out, w4.n_in), torch, device)
+    wo = torch.empty_like(wt)
+    ws = torch.empty(H.workspace_bytes(w4.n_out, w4.n_in), dtype=torch.uint8, device=device)
+    for _ in range(2):
+        H.apply_two_sided(pu, pv, wt, wo, ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st = 3
+    e0.record(stream)
+    for _ in range(st):
+        H.apply_two_sided(pu, pv, wt, wo, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / st
+    b4 = 2 * (2 * w4.n_out * w4.n_in * 2)        # two passes, each reading and writing W once
+    out.append({"workload": WORKLOAD_TEXT["c4"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
+                "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided (4 launches)"})
+    del wt, wo, ws
+    return out
 
 
 def run_ours(args):
@@ -388,19 +444,7 @@ def run_ours(args):
 
     also = []
     if not args.no_extra and rank == 0 and world == 1:
-        for name in ("c3_64k", "c5"):
-            ww = W.get(name)
-            p2 = make_plan(name, H, W)
-            e2 = W.draw_encoded(ww, 0, ww.rows)
-            x2 = to_device_bf16(e2, torch, device)
-            y2 = torch.empty_like(x2)
-            st = max(3, args.steps // 4)
-            el, km, _, kn = time_apply(p2, x2, y2, st, max(3, args.warmup // 2), torch)
-            b2 = 2 * ww.rows * ww.d * 2
-            also.append({"workload": WORKLOAD_TEXT[name], "rows_per_s": ww.rows * st / (el / 1e3),
-                         "hbm_gbs": b2 / (km / 1e3) / 1e9, "hbm_frac": b2 / (km / 1e3) / 1e9 / peak,
-                         "kernel": kn, "kernel_ms": km})
-            del x2, y2, p2
+        also = side_measurements(args, H, W, torch, device, peak)
 
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and world == 1:
