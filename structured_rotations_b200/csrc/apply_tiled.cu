@@ -12,6 +12,29 @@
 
 namespace {
 
+harp_tiled::FastDiv make_fast_div(int n) {
+    harp_tiled::FastDiv f;
+    int l = 0;
+    while ((1ll << l) < n) ++l;
+    f.l = l;
+    f.n = n;
+    f.m = (uint32_t)(((1ull << (32 + l)) + (uint64_t)n - 1) / (uint64_t)n - (1ull << 32));
+    return f;
+}
+
+// Granlund and Montgomery's round-up method ("Division by invariant integers using
+// multiplication", 1994, section 4) makes the quotient exact for every 32-bit x when the
+// 33-bit sum umulhi(x, m) + x is kept; the kernel divides only x < 2^21, so the sum fits in
+// 32 bits.  A cheap check at the edges guards the constants.
+bool fast_div_ok(const harp_tiled::FastDiv& f) {
+    auto q = [&](uint64_t x) { return (uint32_t)(((((uint64_t)x * f.m) >> 32) + x) >> f.l); };
+    const uint64_t n = (uint64_t)f.n;
+    const uint64_t xs[] = {0, 1, n - 1, n, n + 1, 2 * n - 1, ((uint64_t)1 << 21) - 1};
+    for (uint64_t x : xs)
+        if (q(x) != x / n) return false;
+    return true;
+}
+
 int sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -84,17 +107,28 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.staged_rows = (int)staged;
     tp.mask = (d % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
+    for (int t = 0; t < p->desc.m; ++t) {
+        tp.nb_div[t] = make_fast_div((int)p->desc.st[t].nblocks);
+        tp.s_div[t] = make_fast_div((int)p->desc.st[t].s);
+        if (!fast_div_ok(tp.nb_div[t]) || !fast_div_ok(tp.s_div[t])) return HARP_ERR_UNSUPPORTED;
+    }
     const size_t smem = (size_t)R * d * 4 + (size_t)staged * d * es_in + 16;
     const int grid = (int)std::min<int64_t>(tp.ntiles, sm_count());
+    int nt = kThreadChoices[1];
+    {
+        const int qv = (int)((std::min<int64_t>(R, rows) + V - 1) / V);
+        for (int t = 0; t < p->desc.m; ++t)
+            if (stage_groups((int)p->desc.st[t].nblocks, qv, kThreadChoices[1]) > 1) nt = kThreadChoices[0];
+    }
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;
     cudaError_t e;
     if (in_dtype == HARP_BF16 && out_dtype == HARP_BF16)
-        e = harp_tiled_launch_bf16(which, V, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16(which, V, nt, inv, tp, smem, grid, s);
     else if (in_dtype == HARP_F32)
-        e = harp_tiled_launch_f32(which, V, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_f32(which, V, nt, inv, tp, smem, grid, s);
     else
-        e = harp_tiled_launch_bf16_f32(which, V, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16_f32(which, V, nt, inv, tp, smem, grid, s);
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_tiled_kernel");
     return HARP_OK;

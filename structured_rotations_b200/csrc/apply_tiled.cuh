@@ -12,8 +12,8 @@
 // Stage t: each thread takes whole groups {lo + s_t (k + b_t hi)} (block c = lo +
 // s_t hi), holds the block B_{t,c} (b_t x b_t fp32, plain FMA arithmetic) in
 // registers and applies it to every row of the tile, so a block is fetched from L2
-// once per tile rather than once per row; the next block's coefficients are loaded
-// while the current one is applied.  The inverse runs the stages backwards with
+// once per tile rather than once per row; 8 warps per SM hide the load latency.  The
+// inverse runs the stages backwards with
 // B^T (the signs S are folded into stage 0's blocks, so B_0^T also applies S last).
 //
 // Shared-memory layout: the tile is a stack of sub-tiles of V = 4 rows; inside one,
@@ -35,10 +35,21 @@
 
 namespace harp_tiled {
 
-constexpr int kThreads = 256;
 constexpr int kMaxTileRows = 32;
 constexpr int kSmemOptIn = 227 * 1024;
 constexpr long long kWaitLimit = 1ll << 26;   // mbarrier polls before giving up
+
+// Division by a constant n >= 1 of x < 2^21 by multiply and shift: with l = ceil(log2 n)
+// and m = ceil(2^(32+l) / n) - 2^32, x / n = (umulhi(x, m) + x) >> l (built on the host,
+// see make_fast_div).
+struct FastDiv {
+    uint32_t m;
+    int l;
+    int n;
+#ifdef __CUDACC__
+    __device__ __forceinline__ int div(int x) const { return (int)((__umulhi((uint32_t)x, m) + (uint32_t)x) >> l); }
+#endif
+};
 
 struct TiledParams {
     PlanDesc pd;
@@ -52,6 +63,8 @@ struct TiledParams {
     int staged_rows;            // the first rows of the next tile that arrive by bulk copy
     int mask;                   // V = 1 swizzle: 0x18 when d % 32 == 0, else 0
     int* status;
+    FastDiv nb_div[HARP_MAX_STAGES];   // division by d / b_t
+    FastDiv s_div[HARP_MAX_STAGES];    // division by s_t
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -162,26 +175,6 @@ __device__ __forceinline__ void load_block(float (&w)[64], const float* __restri
     }
 }
 
-// The same for a radix known only at run time (the first block of the next stage).
-__device__ __forceinline__ void load_block_any(float (&w)[64], const float* __restrict__ stage, int c, int bb) {
-    const int group = c >> 5, lane = c & 31;
-    if ((bb & 3) == 0) {
-        const float4* src = (const float4*)stage + (size_t)group * (bb / 4) * 32 + lane;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            if (4 * q < bb) {
-                const float4 v = __ldg(src + q * 32);
-                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-            }
-        }
-    } else {
-        const float* src = stage + (size_t)group * bb * 32 + lane;
-#pragma unroll
-        for (int e = 0; e < 64; ++e)
-            if (e < bb) w[e] = __ldg(src + e * 32);
-    }
-}
-
 __device__ __forceinline__ void fma_v(float4& acc, float w, const float4& x) {
     acc.x = fmaf(w, x.x, acc.x);
     acc.y = fmaf(w, x.y, acc.y);
@@ -230,85 +223,56 @@ __device__ __forceinline__ void apply_item(typename VecOf<V>::T* tile, int d, in
 
 // Sub-tile groups of a stage: split the tile's sub-tiles over more items only while
 // too few items would leave a fifth or more of the threads' slots empty.
-__device__ __forceinline__ int stage_groups(int nb, int qv) {
+__host__ __device__ __forceinline__ int stage_groups(int nb, int qv, int nthreads) {
     int G = 1;
     while (G < qv) {
         const int items = nb * G;
-        const int per = (items + kThreads - 1) / kThreads;
-        if (per * kThreads * 4 <= items * 5) break;
+        const int per = (items + nthreads - 1) / nthreads;
+        if (per * nthreads * 4 <= items * 5) break;
         ++G;
     }
     return G;
 }
 
-// What a thread prefetches after its last item of a stage: the first block it will
-// apply in the next stage (of this tile, or stage 0 of its next tile).
-struct NextFirst {
-    const float* stage;   // lane-interleaved blocks of that stage (nullptr: nothing)
-    int nb, bb;
-};
-
-// All items of one stage.  Coefficients are double-buffered in wa / wb: on entry the
-// buffer named by cur_a holds (or is loading) the thread's first block of this stage;
-// while an item is applied the other buffer loads the next one, which after the last
-// item is the first block of the next stage, so on exit cur_a names that buffer.
-template <int B, bool INV, int V>
-__device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, typename VecOf<V>::T* tile,
-                                          int d, int qv, int mask, float (&wa)[64], float (&wb)[64],
-                                          bool& cur_a, const NextFirst& nx) {
+// All items of one stage: items j = tid, tid + T, ...; item j is block c = j % nb of the
+// sub-tiles g = j / nb, g + G, ...  The block's coefficients are loaded into registers at
+// the start of the item (a second register buffer to prefetch the next block costs more
+// in register moves than it saves in latency at 8 warps per SM).
+template <int B, bool INV, int V, int NT>
+__device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, const FastDiv& nbd,
+                                          const FastDiv& sdv, typename VecOf<V>::T* tile, int d, int qv,
+                                          int mask) {
     const int nb = d / B;
-    const int G = stage_groups(nb, qv);
+    const int G = stage_groups(nb, qv, NT);
     const int items = nb * G;
     const int tid = threadIdx.x;
-    int j = tid;
-    if (j >= items) {   // idle in this stage: start loading the next stage's block now
-        if (nx.stage) {
-            if (cur_a) load_block_any(wa, nx.stage, tid % nx.nb, nx.bb);
-            else load_block_any(wb, nx.stage, tid % nx.nb, nx.bb);
-        }
-        return;
-    }
-    // Items j = tid, tid + T, ...: c = j % nb, g = j / nb, and for the block lo = c % s,
-    // hi = c / s, stepped by T without dividing (T % s, T / s once per stage).
+    if (tid >= items) return;
+    // (c, g, lo = c % s, hi = c / s) stepped by T from item to item
     ItemPos it;
-    it.c = tid % nb;
-    it.g = tid / nb;
-    it.lo = it.c % s;
-    it.hi = it.c / s;
-    const int dlo = kThreads % s, dhi = kThreads / s;
-    while (true) {
-        const int jn = j + kThreads;
-        ItemPos nt = it;
-        nt.c += kThreads;
-        nt.lo += dlo;
-        nt.hi += dhi;
-        if (nt.lo >= s) {
-            nt.lo -= s;
-            ++nt.hi;
+    it.g = nbd.div(tid);
+    it.c = tid - nb * it.g;
+    it.hi = sdv.div(it.c);
+    it.lo = it.c - s * it.hi;
+    const int dhi = sdv.div(NT), dlo = NT - s * dhi;
+    float w[64];
+    for (int j = tid; j < items; j += NT) {
+        load_block<B>(w, sb, it.c);
+        apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, w);
+        it.c += NT;
+        it.lo += dlo;
+        it.hi += dhi;
+        if (it.lo >= s) {
+            it.lo -= s;
+            ++it.hi;
         }
-        if (nt.c >= nb) {   // wrapped into the next sub-tile group (small nb only)
-            nt.c -= nb;
-            ++nt.g;
-            while (nt.c >= nb) {
-                nt.c -= nb;
-                ++nt.g;
-            }
-            nt.lo = nt.c % s;
-            nt.hi = nt.c / s;
+        if (it.c >= nb) {   // wrapped into the next sub-tile group (small nb only)
+            do {
+                it.c -= nb;
+                ++it.g;
+            } while (it.c >= nb);
+            it.hi = sdv.div(it.c);
+            it.lo = it.c - s * it.hi;
         }
-        if (cur_a) {
-            if (jn < items) load_block<B>(wb, sb, nt.c);
-            else if (nx.stage) load_block_any(wb, nx.stage, tid % nx.nb, nx.bb);
-            apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, wa);
-        } else {
-            if (jn < items) load_block<B>(wa, sb, nt.c);
-            else if (nx.stage) load_block_any(wa, nx.stage, tid % nx.nb, nx.bb);
-            apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, wb);
-        }
-        cur_a = !cur_a;
-        if (jn >= items) break;
-        j = jn;
-        it = nt;
     }
 }
 
@@ -328,76 +292,90 @@ __device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, u
 // sub-tile and writes them as 8 quads.  V = 1: 8 consecutive coordinates of one row, two
 // 16-byte stores (the XOR keeps 8-aligned runs contiguous).  Rows past the end of the
 // batch are zero.
-template <int V, typename TIn>
+template <int V, int NT, typename TIn>
 __device__ __forceinline__ void fill_tile(typename VecOf<V>::T* tile, int d, int nr, int n_staged, const TIn* staged,
                                           const TIn* src, int64_t ld, int mask) {
     const int d8 = d / 8;
     // row r of the tile: the staging area for r < n_staged, else global memory
     auto row_ptr = [&](int r) -> const TIn* { return r < n_staged ? staged + (size_t)r * d : src + r * ld; };
-    for (int q = 0; V * q < nr; ++q)
-        for (int j = threadIdx.x; j < d8; j += kThreads) {
-            if constexpr (V == 4) {
+    for (int q = 0; V * q < nr; ++q) {
+        if constexpr (V == 4) {
+            const TIn* rp[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rp[e] = row_ptr(min(4 * q + e, nr - 1));
+            float4* st = tile + q * d;
+            for (int j = threadIdx.x; j < d8; j += NT) {
                 float v[4][8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    if (4 * q + e < nr) {
-                        load8(row_ptr(4 * q + e) + 8 * j, v[e]);
-                    } else {
+                    load8(rp[e] + 8 * j, v[e]);
+                    if (4 * q + e >= nr) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k) v[e][k] = 0.0f;
                     }
                 }
-                float4* st = tile + q * d;
+                const int jx = j & 7;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) st[slot<4>(8 * j + k, mask)] = make_float4(v[0][k], v[1][k], v[2][k], v[3][k]);
-            } else {
+                for (int k = 0; k < 8; ++k) st[8 * j + (k ^ jx)] = make_float4(v[0][k], v[1][k], v[2][k], v[3][k]);
+            }
+        } else {
+            const TIn* rp = row_ptr(q);
+            for (int j = threadIdx.x; j < d8; j += NT) {
                 float v[8];
-                load8(row_ptr(q) + 8 * j, v);
+                load8(rp + 8 * j, v);
                 store8(tile + q * d + slot<1>(8 * j, mask), v);
             }
         }
+    }
 }
 
-template <int V, typename TOut>
+template <int V, int NT, typename TOut>
 __device__ __forceinline__ void drain_tile(const typename VecOf<V>::T* tile, int d, int nr, TOut* dst, int64_t ld,
                                            int mask) {
     const int d8 = d / 8;
-    for (int q = 0; V * q < nr; ++q)
-        for (int j = threadIdx.x; j < d8; j += kThreads) {
-            if constexpr (V == 4) {
-                const float4* st = tile + q * d;
+    for (int q = 0; V * q < nr; ++q) {
+        if constexpr (V == 4) {
+            const float4* st = tile + q * d;
+            TOut* rp = dst + (4 * q) * ld;
+            const int rows = min(4, nr - 4 * q);
+            for (int j = threadIdx.x; j < d8; j += NT) {
+                const int jx = j & 7;
                 float4 v4[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) v4[k] = st[slot<4>(8 * j + k, mask)];
+                for (int k = 0; k < 8; ++k) v4[k] = st[8 * j + (k ^ jx)];
                 float v[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) v[k] = v4[k].x;
-                store8(dst + (4 * q) * ld + 8 * j, v);
-                if (4 * q + 1 < nr) {
+                store8(rp + 8 * j, v);
+                if (rows > 1) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) v[k] = v4[k].y;
-                    store8(dst + (4 * q + 1) * ld + 8 * j, v);
+                    store8(rp + ld + 8 * j, v);
                 }
-                if (4 * q + 2 < nr) {
+                if (rows > 2) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) v[k] = v4[k].z;
-                    store8(dst + (4 * q + 2) * ld + 8 * j, v);
+                    store8(rp + 2 * ld + 8 * j, v);
                 }
-                if (4 * q + 3 < nr) {
+                if (rows > 3) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) v[k] = v4[k].w;
-                    store8(dst + (4 * q + 3) * ld + 8 * j, v);
+                    store8(rp + 3 * ld + 8 * j, v);
                 }
-            } else {
+            }
+        } else {
+            TOut* rp = dst + q * ld;
+            for (int j = threadIdx.x; j < d8; j += NT) {
                 float v[8];
                 load8(tile + q * d + slot<1>(8 * j, mask), v);
-                store8(dst + q * ld + 8 * j, v);
+                store8(rp + 8 * j, v);
             }
         }
+    }
 }
 
-template <typename TIn, typename TOut, bool INV, int MASK, int V>
-__global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_constant__ TiledParams p) {
+template <typename TIn, typename TOut, bool INV, int MASK, int V, int NT>
+__global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant__ TiledParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     using VT = typename VecOf<V>::T;
     const int d = (int)p.pd.d;
@@ -417,22 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
     }
     // The stage order: forward 0..m-1, inverse m-1..0.
     auto stage_of = [&](int step) { return INV ? m - 1 - step : step; };
-    auto first_of = [&](int step, int qv_) {
-        const int t = stage_of(step);
-        const int b = p.pd.st[t].b, nb = d / b;
-        NextFirst f;
-        f.stage = tid < nb * stage_groups(nb, qv_) ? p.lanes + p.lane_off[t] : nullptr;
-        f.nb = nb;
-        f.bb = b * b;
-        return f;
-    };
-    float wa[64], wb[64];
-    bool cur_a = true;
-    {
-        const int nr0 = (int)min((int64_t)R, p.rows - t_idx * R);
-        const NextFirst f = first_of(0, (nr0 + V - 1) / V);
-        if (f.stage) load_block_any(wa, f.stage, tid % f.nb, f.bb);
-    }
     uint32_t parity = 0;
     for (; t_idx < p.ntiles; t_idx += gridDim.x) {
         const int64_t row0 = t_idx * R;
@@ -447,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
                 return;
             }
         }
-        fill_tile<V, TIn>(tile, d, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x, p.ld_x,
+        fill_tile<V, NT, TIn>(tile, d, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x, p.ld_x,
                           p.mask);
         __syncthreads();
         const int64_t t_next = t_idx + gridDim.x;
@@ -455,20 +417,16 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
             fence_proxy_async_smem();   // the staging reads above happen before the copies' writes
             issue_tile<TIn>(p, t_next, stage_buf, bar);
         }
-        const int nr_next = t_next < p.ntiles ? (int)min((int64_t)R, p.rows - t_next * R) : 0;
         for (int step = 0; step < m; ++step) {
             const int t = stage_of(step);
             const StageDesc& sd = p.pd.st[t];
-            NextFirst nx;
-            if (step + 1 < m) nx = first_of(step + 1, qv);
-            else if (nr_next) nx = first_of(0, (nr_next + V - 1) / V);
-            else nx.stage = nullptr, nx.nb = 1, nx.bb = 0;
             const float* sb = p.lanes + p.lane_off[t];
             const int s = (int)sd.s;
             switch (sd.b) {
-#define HARP_TILED_CASE(R)                                                                       \
-    case R:                                                                                      \
-        if constexpr ((MASK >> R) & 1) run_stage<R, INV, V>(sb, s, tile, d, qv, p.mask, wa, wb, cur_a, nx); \
+#define HARP_TILED_CASE(R)                                                                          \
+    case R:                                                                                         \
+        if constexpr ((MASK >> R) & 1)                                                              \
+            run_stage<R, INV, V, NT>(sb, s, p.nb_div[t], p.s_div[t], tile, d, qv, p.mask);          \
         break;
                 HARP_TILED_CASE(2) HARP_TILED_CASE(3) HARP_TILED_CASE(4) HARP_TILED_CASE(5)
                 HARP_TILED_CASE(6) HARP_TILED_CASE(7) HARP_TILED_CASE(8)
@@ -477,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) harp_tiled_kernel(const __grid_co
             }
             __syncthreads();
         }
-        drain_tile<V, TOut>(tile, d, nr, (TOut*)p.y + row0 * p.ld_y, p.ld_y, p.mask);
+        drain_tile<V, NT, TOut>(tile, d, nr, (TOut*)p.y + row0 * p.ld_y, p.ld_y, p.mask);
         __syncthreads();
     }
 }
@@ -493,17 +451,21 @@ constexpr int kNumMasks = sizeof(kMasks) / sizeof(kMasks[0]);
 // memory (d > 14524); they are built for the radix sets without 5.
 constexpr bool has_row_major_kernel(int mask) { return ((mask >> 5) & 1) == 0; }
 
-template <typename TIn, typename TOut, bool INV, int V, int I>
+// Threads per CTA: 384 (12 warps, at most 168 registers) when every stage splits evenly
+// over them without dividing the tile's sub-tiles between items; else 256.
+constexpr int kThreadChoices[] = {256, 384};
+
+template <typename TIn, typename TOut, bool INV, int V, int NT, int I>
 cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
     if constexpr (I < kNumMasks) {
-        if (which != I) return launch_mask<TIn, TOut, INV, V, I + 1>(which, tp, smem, grid, stream);
+        if (which != I) return launch_mask<TIn, TOut, INV, V, NT, I + 1>(which, tp, smem, grid, stream);
         if constexpr (V == 1 && !has_row_major_kernel(kMasks[I])) {
             return cudaErrorInvalidValue;
         } else {
-            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V>;
+            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT>;
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            kern<<<(unsigned)grid, kThreads, smem, stream>>>(tp);
+            kern<<<(unsigned)grid, NT, smem, stream>>>(tp);
             return cudaGetLastError();
         }
     } else {
@@ -511,22 +473,28 @@ cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid,
     }
 }
 
+template <typename TIn, typename TOut, bool INV, int V>
+cudaError_t launch_nt(int which, int nt, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
+    if (nt == 384) return launch_mask<TIn, TOut, INV, V, 384, 0>(which, tp, smem, grid, stream);
+    return launch_mask<TIn, TOut, INV, V, 256, 0>(which, tp, smem, grid, stream);
+}
+
 template <typename TIn, typename TOut>
-cudaError_t launch(int which, int V, bool inverse, const TiledParams& tp, size_t smem, int grid,
+cudaError_t launch(int which, int V, int nt, bool inverse, const TiledParams& tp, size_t smem, int grid,
                    cudaStream_t stream) {
     if (V == 4)
-        return inverse ? launch_mask<TIn, TOut, true, 4, 0>(which, tp, smem, grid, stream)
-                       : launch_mask<TIn, TOut, false, 4, 0>(which, tp, smem, grid, stream);
-    return inverse ? launch_mask<TIn, TOut, true, 1, 0>(which, tp, smem, grid, stream)
-                   : launch_mask<TIn, TOut, false, 1, 0>(which, tp, smem, grid, stream);
+        return inverse ? launch_nt<TIn, TOut, true, 4>(which, nt, tp, smem, grid, stream)
+                       : launch_nt<TIn, TOut, false, 4>(which, nt, tp, smem, grid, stream);
+    return inverse ? launch_nt<TIn, TOut, true, 1>(which, nt, tp, smem, grid, stream)
+                   : launch_nt<TIn, TOut, false, 1>(which, nt, tp, smem, grid, stream);
 }
 
 }  // namespace harp_tiled
 
 // One translation unit per I/O type pair (compiled in parallel).
-cudaError_t harp_tiled_launch_bf16(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_bf16(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
                                    size_t smem, int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_f32(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_f32(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
                                   size_t smem, int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_bf16_f32(int which, int V, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_bf16_f32(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
                                        size_t smem, int grid, cudaStream_t stream);
