@@ -125,9 +125,15 @@ extern "C" harp_status harp_apply_two_sided(harp_plan_t pu, harp_plan_t pv, cons
     // rows of W: w_r <- T_V^T w_r (fp32 out)
     st = run_rows(pv, W, ws1, n_out, ld, n_in, dtype, HARP_F32, HARP_INVERSE, stream);
     if (st != HARP_OK) return st;
+    // columns: col <- T_U^T col, in two passes over ws1, the second writing W_out
+    if (kernel_choice() != kSimple) {
+        st = launch_cols(pu, ws1, n_in, n_in, W_out, ld, dtype, HARP_INVERSE, stream);
+        if (st != HARP_ERR_UNSUPPORTED) return st;
+        harp_clear_error();
+    }
+    // otherwise: transpose, rows of W^T, transpose back
     if ((st = launch_transpose(ws1, ws2, n_out, n_in, n_in, n_out, HARP_F32, HARP_F32, stream)) != HARP_OK)
         return st;
-    // columns of W (rows of W^T): col <- T_U^T col
     st = run_rows(pu, ws2, ws2, n_in, n_out, n_out, HARP_F32, HARP_F32, HARP_INVERSE, stream);
     if (st != HARP_OK) return st;
     return launch_transpose(ws2, W_out, n_in, n_out, n_out, ld, HARP_F32, dtype, stream);

@@ -1,0 +1,260 @@
+// Column passes of the two-sided rotation (HARP abstract: a rotation on each side of a
+// weight matrix): every column of an fp32 matrix X with d rows takes T or T^T of one
+// plan, with the result written in place or rounded to the output type.
+//
+// Stage t mixes the rows {lo + s_t (k + b_t hi)} of X with block B_{t,c}, the same
+// b_t x b_t block for every column.  So a block is loaded once per tile and serves all
+// of its 64 columns (the 32 lanes of a warp hold 2 columns each and load the block's
+// coefficients with warp-uniform addresses, a broadcast), and the columns never need a
+// transpose.
+//
+// The stages split at t* into two passes over X (P = s_{t*} = prod_{t<t*} b_t, Q = d / P):
+//  - pass A, stages t >= t*: for fixed p in [0, P) the rows {p + P v : v < Q} form a
+//    Q-coordinate problem in v, where stage t has stride s_t / P and the block of local
+//    index c_v is c = p + P c_v.  A tile holds PB consecutive p values, PB*Q rows.
+//  - pass B, stages t < t*: a slab of P contiguous rows; the block of local index c_l
+//    in slab n is c = n (P / b_t) + c_l.
+// The inverse runs pass A (stages m-1 .. t*) then pass B (t*-1 .. 0) with transposed
+// blocks; the forward direction runs pass B (0 .. t*-1) then pass A (t* .. m-1).
+#include <algorithm>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "harp_internal.h"
+
+namespace {
+
+constexpr int kCols = 64;          // columns per tile: 2 per lane
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct ColsParams {
+    PlanDesc pd;
+    const float* blocks;   // row-major [stage][c][k][l]
+    float* x;              // d rows, leading dimension ld_x (fp32)
+    void* y;               // output rows (== x for in place), leading dimension ld_y
+    int64_t ld_x, ld_y;
+    int ncols;
+    int pass_a;            // 1: row sets {p + P v}; 0: slabs of P rows
+    int P, Q, PB, SB;      // PB p values per pass-A tile, SB slabs per pass-B tile
+    int t_first, t_last, t_step;   // stages t_first, t_first + t_step, ..., t_last
+    int inverse;
+    int out_bf16;
+};
+
+__device__ __forceinline__ int tile_row_global(const ColsParams& p, int tile_r, int i) {
+    // pass A: tile tile_r covers p = tile_r * PB + pb, its row i = pb * Q + v;
+    // pass B: tile tile_r covers slabs tile_r * SB ..., contiguous rows
+    if (p.pass_a) {
+        const int pb = i / p.Q, v = i - pb * p.Q;
+        return tile_r * p.PB + pb + p.P * v;
+    }
+    return tile_r * p.SB * p.P + i;
+}
+
+template <int B>
+__device__ __forceinline__ void apply_group(float2* __restrict__ tile, const ColsParams& p, const float* blk,
+                                            bool vec, const int (&rows)[B], int lane) {
+    float w[B * B];
+    bool done = false;
+    if constexpr ((B * B) % 4 == 0) {
+        if (vec) {   // 16-byte aligned block
+#pragma unroll
+            for (int q = 0; q < B * B / 4; ++q) {
+                const float4 v = __ldg((const float4*)blk + q);
+                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+            }
+            done = true;
+        }
+    }
+    if (!done) {
+#pragma unroll
+        for (int e = 0; e < B * B; ++e) w[e] = __ldg(blk + e);
+    }
+    float2 xv[B];
+#pragma unroll
+    for (int l = 0; l < B; ++l) xv[l] = tile[rows[l] * (kCols / 2) + lane];
+    float2 yv[B];
+#pragma unroll
+    for (int k = 0; k < B; ++k) yv[k] = make_float2(0.f, 0.f);
+    // every output sums over l = 0..b-1 in order
+#pragma unroll
+    for (int l = 0; l < B; ++l)
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            const float c = p.inverse ? w[l * B + k] : w[k * B + l];
+            yv[k].x = fmaf(c, xv[l].x, yv[k].x);
+            yv[k].y = fmaf(c, xv[l].y, yv[k].y);
+        }
+#pragma unroll
+    for (int k = 0; k < B; ++k) tile[rows[k] * (kCols / 2) + lane] = yv[k];
+}
+
+template <int B>
+__device__ __forceinline__ void run_stage(float2* tile, const ColsParams& p, const StageDesc& sd, int tile_r,
+                                          int warp, int lane) {
+    // local stride and block count of one problem (a p value in pass A, the slab in B)
+    const int sl = p.pass_a ? (int)(sd.s / p.P) : (int)sd.s;
+    const int n_local = (p.pass_a ? p.Q : p.P) / B;          // blocks of one problem
+    const int n_items = (p.pass_a ? p.PB : p.SB) * n_local;
+    for (int item = warp; item < n_items; item += kWarps) {
+        const int pb = item / n_local, cl = item - pb * n_local;   // problem, local block
+        const int lo = cl % sl, hi = cl / sl;
+        const int base = pb * (p.pass_a ? p.Q : p.P) + lo + sl * B * hi;
+        int rows[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k) rows[k] = base + sl * k;
+        const int64_t c = p.pass_a ? (int64_t)(tile_r * p.PB + pb) + (int64_t)p.P * cl
+                                   : (int64_t)(tile_r * p.SB + pb) * (p.P / B) + cl;
+        apply_group<B>(tile, p, p.blocks + sd.block_off + c * (B * B), (sd.block_off & 3) == 0, rows, lane);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) harp_cols_kernel(const __grid_constant__ ColsParams p) {
+    extern __shared__ __align__(16) float2 tile[];
+    const int rows_per_tile = p.pass_a ? p.PB * p.Q : p.SB * p.P;
+    const int col_tiles = (p.ncols + kCols - 1) / kCols;
+    const int tile_r = blockIdx.x / col_tiles;
+    const int col0 = (blockIdx.x - tile_r * col_tiles) * kCols;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool full = col0 + kCols <= p.ncols;
+
+    // load: 16 float4 per row
+    for (int e = tid; e < rows_per_tile * (kCols / 4); e += kThreads) {
+        const int i = e / (kCols / 4), cq = e - i * (kCols / 4);
+        const float* src = p.x + (int64_t)tile_row_global(p, tile_r, i) * p.ld_x + col0 + 4 * cq;
+        float4 v;
+        if (full) {
+            v = *(const float4*)src;
+        } else {
+            const int c = col0 + 4 * cq;
+            v.x = c < p.ncols ? src[0] : 0.f;
+            v.y = c + 1 < p.ncols ? src[1] : 0.f;
+            v.z = c + 2 < p.ncols ? src[2] : 0.f;
+            v.w = c + 3 < p.ncols ? src[3] : 0.f;
+        }
+        ((float4*)tile)[e] = v;
+    }
+    __syncthreads();
+    for (int t = p.t_first;; t += p.t_step) {
+        const StageDesc& sd = p.pd.st[t];
+        switch (sd.b) {
+            case 2: run_stage<2>(tile, p, sd, tile_r, warp, lane); break;
+            case 3: run_stage<3>(tile, p, sd, tile_r, warp, lane); break;
+            case 4: run_stage<4>(tile, p, sd, tile_r, warp, lane); break;
+            case 5: run_stage<5>(tile, p, sd, tile_r, warp, lane); break;
+            case 6: run_stage<6>(tile, p, sd, tile_r, warp, lane); break;
+            case 7: run_stage<7>(tile, p, sd, tile_r, warp, lane); break;
+            case 8: run_stage<8>(tile, p, sd, tile_r, warp, lane); break;
+            default: break;
+        }
+        __syncthreads();
+        if (t == p.t_last) break;
+    }
+    // store: fp32 (16 bytes per thread) or bf16 (8 bytes)
+    for (int e = tid; e < rows_per_tile * (kCols / 4); e += kThreads) {
+        const int i = e / (kCols / 4), cq = e - i * (kCols / 4);
+        const int64_t row = tile_row_global(p, tile_r, i);
+        const int c = col0 + 4 * cq;
+        const float4 v = ((const float4*)tile)[e];
+        if (p.out_bf16) {
+            __nv_bfloat16* dst = (__nv_bfloat16*)p.y + row * p.ld_y + c;
+            if (full) {
+                const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+                uint2 u;
+                u.x = *(const uint32_t*)&a;
+                u.y = *(const uint32_t*)&b;
+                *(uint2*)dst = u;
+            } else {
+                const float f[4] = {v.x, v.y, v.z, v.w};
+                for (int k = 0; k < 4; ++k)
+                    if (c + k < p.ncols) dst[k] = __float2bfloat16_rn(f[k]);
+            }
+        } else {
+            float* dst = (float*)p.y + row * p.ld_y + c;
+            if (full) {
+                *(float4*)dst = v;
+            } else {
+                const float f[4] = {v.x, v.y, v.z, v.w};
+                for (int k = 0; k < 4; ++k)
+                    if (c + k < p.ncols) dst[k] = f[k];
+            }
+        }
+    }
+}
+
+}  // namespace
+
+// Column transform of an fp32 matrix x (d rows of ncols, leading dimension ld_x) by
+// the plan's T (forward) or T^T (inverse); the result goes to y (fp32 with ld_y, which
+// may be x itself, or bf16).  Two passes, each a kernel launch on `stream`.
+harp_status launch_cols(const harp_plan_s* pl, float* x, int64_t ld_x, int64_t ncols, void* y, int64_t ld_y,
+                        harp_dtype out_dtype, harp_dir dir, void* stream_) {
+    const PlanDesc& pd = pl->desc;
+    const int64_t d = pd.d;
+    if (pd.m < 2 || ncols <= 0 || ncols > (int64_t)1 << 30) return HARP_ERR_UNSUPPORTED;
+    for (int t = 0; t < pd.m; ++t)
+        if (pd.st[t].b > 8) return HARP_ERR_UNSUPPORTED;
+    if (((uintptr_t)x & 15) || (ld_x & 3) || ((uintptr_t)y & 15) || (ld_y & 3)) return HARP_ERR_UNSUPPORTED;
+    // the split t* that keeps both tiles smallest
+    const int64_t row_bytes = kCols * 4;
+    int best = -1;
+    int64_t best_size = 0;
+    for (int t = 1; t < pd.m; ++t) {
+        const int64_t P = pd.st[t].s, Q = d / P;
+        if (P * row_bytes > kSmemBudget || Q * row_bytes > kSmemBudget) continue;
+        const int64_t size = std::max(P, Q);
+        if (best < 0 || size < best_size) best = t, best_size = size;
+    }
+    if (best < 0) return HARP_ERR_UNSUPPORTED;
+    const int P = (int)pd.st[best].s, Q = (int)(d / P);
+    int PB = (int)std::min<int64_t>(P, kSmemBudget / (Q * row_bytes));
+    while (P % PB) --PB;
+    int SB = (int)std::min<int64_t>(Q, kSmemBudget / (P * row_bytes));
+    while (Q % SB) --SB;
+    const int col_tiles = (int)((ncols + kCols - 1) / kCols);
+    cudaStream_t stream = (cudaStream_t)stream_;
+
+    ColsParams cp;
+    cp.pd = pd;
+    cp.blocks = pl->d_blocks;
+    cp.x = x;
+    cp.ld_x = ld_x;
+    cp.ncols = (int)ncols;
+    cp.P = P;
+    cp.Q = Q;
+    cp.PB = PB;
+    cp.SB = SB;
+    cp.inverse = dir == HARP_INVERSE;
+    const bool inv = dir == HARP_INVERSE;
+    for (int pass = 0; pass < 2; ++pass) {
+        // inverse: A (m-1 .. t*) then B (t*-1 .. 0); forward: B (0 .. t*-1) then A (t* .. m-1)
+        const bool a = inv ? pass == 0 : pass == 1;
+        cp.pass_a = a;
+        if (a) {
+            cp.t_first = inv ? pd.m - 1 : best;
+            cp.t_last = inv ? best : pd.m - 1;
+        } else {
+            cp.t_first = inv ? best - 1 : 0;
+            cp.t_last = inv ? 0 : best - 1;
+        }
+        cp.t_step = inv ? -1 : 1;
+        const bool last = pass == 1;
+        cp.y = last ? y : (void*)x;
+        cp.ld_y = last ? ld_y : ld_x;
+        cp.out_bf16 = last && out_dtype == HARP_BF16;
+        const int row_tiles = a ? P / PB : Q / SB;
+        const size_t smem = (size_t)(a ? PB * Q : SB * P) * row_bytes;
+        cudaError_t e = cudaFuncSetAttribute(harp_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+        const int64_t grid = (int64_t)row_tiles * col_tiles;
+        if (grid > 0x7fffffff) return HARP_ERR_UNSUPPORTED;
+        harp_cols_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(cp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    }
+    harp_set_last_kernel("harp_cols_kernel");
+    return HARP_OK;
+}

@@ -80,6 +80,12 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               void* stream, harp_dtype out_dtype);
 void fast_state_free(harp_plan_s* p);
 
+// Column transform for the two-sided rotation (cols.cu): every column of an fp32 matrix
+// x (d rows) takes T (forward) or T^T (inverse); result to y (fp32, may be x, or bf16).
+// HARP_ERR_UNSUPPORTED for schedules it does not cover (radix > 8, one stage, ...).
+harp_status launch_cols(const harp_plan_s* p, float* x, int64_t ld_x, int64_t ncols, void* y, int64_t ld_y,
+                        harp_dtype out_dtype, harp_dir dir, void* stream);
+
 // General tiled row kernel (apply_tiled.cu): radices 2..8, d % 8 == 0, 16-byte aligned
 // rows.  Returns HARP_ERR_UNSUPPORTED for other shapes.
 harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
