@@ -44,6 +44,19 @@ struct ColsParams {
     int out_bf16;
 };
 
+__device__ __forceinline__ uint32_t smem_u32(const void* ptr) {
+    return (uint32_t)__cvta_generic_to_shared(ptr);
+}
+
+// Asynchronous global -> shared copies (no register staging, all in flight at once).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ int tile_row_global(const ColsParams& p, int tile_r, int i) {
     // pass A: tile tile_r covers p = tile_r * PB + pb, its row i = pb * Q + v;
     // pass B: tile tile_r covers slabs tile_r * SB ..., contiguous rows
@@ -54,24 +67,21 @@ __device__ __forceinline__ int tile_row_global(const ColsParams& p, int tile_r, 
     return tile_r * p.SB * p.P + i;
 }
 
+// One group of b rows times the lane's 2 columns; the block comes from the tile's copy
+// in shared memory (every lane reads the same address: a broadcast).
 template <int B>
 __device__ __forceinline__ void apply_group(float2* __restrict__ tile, const ColsParams& p, const float* blk,
-                                            bool vec, const int (&rows)[B], int lane) {
+                                            const int (&rows)[B], int lane) {
     float w[B * B];
-    bool done = false;
     if constexpr ((B * B) % 4 == 0) {
-        if (vec) {   // 16-byte aligned block
 #pragma unroll
-            for (int q = 0; q < B * B / 4; ++q) {
-                const float4 v = __ldg((const float4*)blk + q);
-                w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-            }
-            done = true;
+        for (int q = 0; q < B * B / 4; ++q) {
+            const float4 v = ((const float4*)blk)[q];
+            w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
         }
-    }
-    if (!done) {
+    } else {
 #pragma unroll
-        for (int e = 0; e < B * B; ++e) w[e] = __ldg(blk + e);
+        for (int e = 0; e < B * B; ++e) w[e] = blk[e];
     }
     float2 xv[B];
 #pragma unroll
@@ -93,7 +103,7 @@ __device__ __forceinline__ void apply_group(float2* __restrict__ tile, const Col
 }
 
 template <int B>
-__device__ __forceinline__ void run_stage(float2* tile, const ColsParams& p, const StageDesc& sd, int tile_r,
+__device__ __forceinline__ void run_stage(float2* tile, const float* coef, const ColsParams& p, const StageDesc& sd,
                                           int warp, int lane) {
     // local stride and block count of one problem (a p value in pass A, the slab in B)
     const int sl = p.pass_a ? (int)(sd.s / p.P) : (int)sd.s;
@@ -106,50 +116,90 @@ __device__ __forceinline__ void run_stage(float2* tile, const ColsParams& p, con
         int rows[B];
 #pragma unroll
         for (int k = 0; k < B; ++k) rows[k] = base + sl * k;
-        const int64_t c = p.pass_a ? (int64_t)(tile_r * p.PB + pb) + (int64_t)p.P * cl
-                                   : (int64_t)(tile_r * p.SB + pb) * (p.P / B) + cl;
-        apply_group<B>(tile, p, p.blocks + sd.block_off + c * (B * B), (sd.block_off & 3) == 0, rows, lane);
+        apply_group<B>(tile, p, coef + item * (B * B), rows, lane);
     }
+}
+
+// Items of one stage in a tile: (problem pb, local block cl), item = pb * n_local + cl;
+// the global block index of an item.
+__device__ __forceinline__ int64_t item_block(const ColsParams& p, const StageDesc& sd, int tile_r, int item) {
+    const int n_local = (p.pass_a ? p.Q : p.P) / sd.b;
+    const int pb = item / n_local, cl = item - pb * n_local;
+    return p.pass_a ? (int64_t)(tile_r * p.PB + pb) + (int64_t)p.P * cl
+                    : (int64_t)(tile_r * p.SB + pb) * (p.P / sd.b) + cl;
+}
+
+__device__ __forceinline__ int stage_items(const ColsParams& p, const StageDesc& sd) {
+    return (p.pass_a ? p.PB * p.Q : p.SB * p.P) / sd.b;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) harp_cols_kernel(const __grid_constant__ ColsParams p) {
     extern __shared__ __align__(16) float2 tile[];
     const int rows_per_tile = p.pass_a ? p.PB * p.Q : p.SB * p.P;
+    float* coef = (float*)(tile + rows_per_tile * (kCols / 2));
     const int col_tiles = (p.ncols + kCols - 1) / kCols;
     const int tile_r = blockIdx.x / col_tiles;
     const int col0 = (blockIdx.x - tile_r * col_tiles) * kCols;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool full = col0 + kCols <= p.ncols;
 
+    // the blocks of every stage of this pass that the tile's groups use, stage after
+    // stage (each stage's part starts on a 16-byte boundary), item order
+    {
+        int off = 0;
+        for (int t = p.t_first;; t += p.t_step) {
+            const StageDesc& sd = p.pd.st[t];
+            const int bb = sd.b * sd.b, n = stage_items(p, sd) * bb;
+            if ((bb & 3) == 0 && (sd.block_off & 3) == 0) {   // whole 16-byte pieces
+                const int bb4 = bb / 4;
+                for (int e = tid; e < n / 4; e += kThreads) {
+                    const int item = e / bb4, k = e - item * bb4;
+                    cp_async16(coef + off + 4 * e,
+                               p.blocks + sd.block_off + item_block(p, sd, tile_r, item) * bb + 4 * k);
+                }
+            } else {
+                for (int e = tid; e < n; e += kThreads) {
+                    const int item = e / bb, k = e - item * bb;
+                    cp_async4(coef + off + e, p.blocks + sd.block_off + item_block(p, sd, tile_r, item) * bb + k);
+                }
+            }
+            off += (n + 3) & ~3;
+            if (t == p.t_last) break;
+        }
+    }
     // load: 16 float4 per row
     for (int e = tid; e < rows_per_tile * (kCols / 4); e += kThreads) {
         const int i = e / (kCols / 4), cq = e - i * (kCols / 4);
         const float* src = p.x + (int64_t)tile_row_global(p, tile_r, i) * p.ld_x + col0 + 4 * cq;
-        float4 v;
         if (full) {
-            v = *(const float4*)src;
+            cp_async16((float4*)tile + e, src);
         } else {
             const int c = col0 + 4 * cq;
+            float4 v;
             v.x = c < p.ncols ? src[0] : 0.f;
             v.y = c + 1 < p.ncols ? src[1] : 0.f;
             v.z = c + 2 < p.ncols ? src[2] : 0.f;
             v.w = c + 3 < p.ncols ? src[3] : 0.f;
+            ((float4*)tile)[e] = v;
         }
-        ((float4*)tile)[e] = v;
     }
+    cp_async_wait_all();
     __syncthreads();
+    int off = 0;
     for (int t = p.t_first;; t += p.t_step) {
         const StageDesc& sd = p.pd.st[t];
+        const float* cs = coef + off;
         switch (sd.b) {
-            case 2: run_stage<2>(tile, p, sd, tile_r, warp, lane); break;
-            case 3: run_stage<3>(tile, p, sd, tile_r, warp, lane); break;
-            case 4: run_stage<4>(tile, p, sd, tile_r, warp, lane); break;
-            case 5: run_stage<5>(tile, p, sd, tile_r, warp, lane); break;
-            case 6: run_stage<6>(tile, p, sd, tile_r, warp, lane); break;
-            case 7: run_stage<7>(tile, p, sd, tile_r, warp, lane); break;
-            case 8: run_stage<8>(tile, p, sd, tile_r, warp, lane); break;
+            case 2: run_stage<2>(tile, cs, p, sd, warp, lane); break;
+            case 3: run_stage<3>(tile, cs, p, sd, warp, lane); break;
+            case 4: run_stage<4>(tile, cs, p, sd, warp, lane); break;
+            case 5: run_stage<5>(tile, cs, p, sd, warp, lane); break;
+            case 6: run_stage<6>(tile, cs, p, sd, warp, lane); break;
+            case 7: run_stage<7>(tile, cs, p, sd, warp, lane); break;
+            case 8: run_stage<8>(tile, cs, p, sd, warp, lane); break;
             default: break;
         }
+        off += (stage_items(p, sd) * sd.b * sd.b + 3) & ~3;
         __syncthreads();
         if (t == p.t_last) break;
     }
@@ -198,21 +248,29 @@ harp_status launch_cols(const harp_plan_s* pl, float* x, int64_t ld_x, int64_t n
     for (int t = 0; t < pd.m; ++t)
         if (pd.st[t].b > 8) return HARP_ERR_UNSUPPORTED;
     if (((uintptr_t)x & 15) || (ld_x & 3) || ((uintptr_t)y & 15) || (ld_y & 3)) return HARP_ERR_UNSUPPORTED;
-    // the split t* that keeps both tiles smallest
-    const int64_t row_bytes = kCols * 4;
+    // Split t*: a tile row costs 256 bytes of data plus 4 sum_t b_t bytes of the blocks
+    // of its pass's stages; pick the split whose larger problem (P or Q rows) is smallest.
+    const int64_t data_row = kCols * 4;
+    auto coef_row = [&](int t0, int t1) {   // bytes of blocks per tile row, stages [t0, t1)
+        int64_t s4 = 0;
+        for (int t = t0; t < t1; ++t) s4 += 4 * pd.st[t].b + 16;
+        return s4;
+    };
     int best = -1;
     int64_t best_size = 0;
     for (int t = 1; t < pd.m; ++t) {
         const int64_t P = pd.st[t].s, Q = d / P;
-        if (P * row_bytes > kSmemBudget || Q * row_bytes > kSmemBudget) continue;
+        if (P * (data_row + coef_row(0, t)) > kSmemBudget || Q * (data_row + coef_row(t, pd.m)) > kSmemBudget)
+            continue;
         const int64_t size = std::max(P, Q);
         if (best < 0 || size < best_size) best = t, best_size = size;
     }
     if (best < 0) return HARP_ERR_UNSUPPORTED;
     const int P = (int)pd.st[best].s, Q = (int)(d / P);
-    int PB = (int)std::min<int64_t>(P, kSmemBudget / (Q * row_bytes));
+    const int64_t row_a = data_row + coef_row(best, pd.m), row_b = data_row + coef_row(0, best);
+    int PB = (int)std::min<int64_t>(P, kSmemBudget / (Q * row_a));
     while (P % PB) --PB;
-    int SB = (int)std::min<int64_t>(Q, kSmemBudget / (P * row_bytes));
+    int SB = (int)std::min<int64_t>(Q, kSmemBudget / (P * row_b));
     while (Q % SB) --SB;
     const int col_tiles = (int)((ncols + kCols - 1) / kCols);
     cudaStream_t stream = (cudaStream_t)stream_;
@@ -246,7 +304,7 @@ harp_status launch_cols(const harp_plan_s* pl, float* x, int64_t ld_x, int64_t n
         cp.ld_y = last ? ld_y : ld_x;
         cp.out_bf16 = last && out_dtype == HARP_BF16;
         const int row_tiles = a ? P / PB : Q / SB;
-        const size_t smem = (size_t)(a ? PB * Q : SB * P) * row_bytes;
+        const size_t smem = (size_t)(a ? PB * Q * row_a : SB * P * row_b);
         cudaError_t e = cudaFuncSetAttribute(harp_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
         const int64_t grid = (int64_t)row_tiles * col_tiles;
