@@ -3,6 +3,8 @@
 // shared-memory budget, the radix-set instantiation that covers the schedule, and one
 // persistent CTA per SM.
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -72,29 +74,58 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     while (which < kNumMasks && (kMasks[which] & mask) != mask) ++which;
     if (which == kNumMasks) return HARP_ERR_UNSUPPORTED;
 
-    // Rows per tile R = V Q: as many sub-tiles of V = 4 rows (fp32, 16 d bytes each) as fit,
-    // then as many of the next tile's raw rows as fit in the rest go to a staging area
-    // (bulk copies overlap the arithmetic; the other rows are read directly).  One
-    // sub-tile fewer when that would stage fewer than half the rows.  Sub-tiles of one
-    // row when not even one 4-row sub-tile fits.
+    // Rows per tile R = V Q for a CTA holding dl coordinates of each row: as many sub-tiles
+    // of V = 4 rows (fp32, 16 dl bytes each) as fit, then as many of the next tile's raw
+    // rows as fit in the rest go to a staging area (bulk copies overlap the arithmetic; the
+    // other rows are read directly).  One sub-tile fewer when that would stage fewer than
+    // half the rows.  Sub-tiles of one row when not even one 4-row sub-tile fits.
     const int64_t budget = kSmemOptIn - 64;
-    auto staged_for = [&](int64_t r) {
-        return std::max<int64_t>(0, std::min<int64_t>(r, (budget - r * d * 4) / (d * es_in)));
+    struct Shape {
+        int V;
+        int64_t R, staged;
     };
-    int V = 4;
-    int64_t Q = std::min<int64_t>(budget / (16 * d), kMaxTileRows / 4);
-    if (Q > 1 && staged_for(4 * Q) < 2 * Q) --Q;
-    if (Q < 1) {
-        V = 1;
-        Q = std::min<int64_t>(budget / (4 * d), kMaxTileRows);
-        if (Q < 1 || !has_row_major_kernel(kMasks[which])) return HARP_ERR_UNSUPPORTED;
+    auto shape_for = [&](int64_t dl) -> Shape {
+        auto staged_for = [&](int64_t r) {
+            return std::max<int64_t>(0, std::min<int64_t>(r, (budget - r * dl * 4) / (dl * es_in)));
+        };
+        Shape sh{4, 0, 0};
+        int64_t Q = std::min<int64_t>(budget / (16 * dl), kMaxTileRows / 4);
+        if (Q > 1 && staged_for(4 * Q) < 2 * Q) --Q;
+        if (Q < 1) {
+            sh.V = 1;
+            Q = std::min<int64_t>(budget / (4 * dl), kMaxTileRows);
+        }
+        Q = std::min<int64_t>(Q, (rows + sh.V - 1) / sh.V);
+        sh.R = sh.V * Q;
+        sh.staged = sh.R > 0 ? std::min<int64_t>(staged_for(sh.R), rows) : 0;
+        return sh;
+    };
+    // Slab mode (a cluster of two CTAs, each with half of every row) for schedules whose
+    // last radix is 2, when it doubles the rows per tile.  Opt-in (HARP_TILED_SLAB=1): it
+    // halves the coefficient stream per row but measured no faster than whole rows on
+    // B200 (d = 8192: equal; d = 5120: slower), whose limit here is issue rate.
+    const PlanDesc& pd = p->desc;
+    int cl = 1;
+    Shape sh = shape_for(d);
+    {
+        const char* env = std::getenv("HARP_TILED_SLAB");
+        bool ok = env && !std::strcmp(env, "1") && pd.m >= 2 && pd.st[pd.m - 1].b == 2 && d % 16 == 0 &&
+                  has_slab_kernel(kMasks[which]) && (pd.st[pd.m - 1].block_off & 3) == 0;
+        for (int t = 0; ok && t < pd.m - 1; ++t) ok = ((d / 2) / pd.st[t].b) % 32 == 0;
+        if (ok) {
+            const Shape s2 = shape_for(d / 2);
+            if (s2.V == 4 && s2.R >= 2 * sh.R) {
+                sh = s2;
+                cl = 2;
+            }
+        }
     }
-    Q = std::min<int64_t>(Q, (rows + V - 1) / V);
-    const int64_t R = V * Q;
-    const int64_t staged = std::min<int64_t>(staged_for(R), rows);
+    const int V = sh.V;
+    const int64_t R = sh.R, staged = sh.staged, dl = d / cl;
+    if (R < 1 || (V == 1 && !has_row_major_kernel(kMasks[which]))) return HARP_ERR_UNSUPPORTED;
 
     TiledParams tp;
-    tp.pd = p->desc;
+    tp.pd = pd;
     tp.lanes = p->d_blocks_lanes;
     for (int t = 0; t < HARP_MAX_STAGES; ++t) tp.lane_off[t] = p->lane_off[t];
     tp.x = x;
@@ -105,30 +136,31 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.ntiles = (rows + R - 1) / R;
     tp.R = (int)R;
     tp.staged_rows = (int)staged;
-    tp.mask = (d % 32 == 0) ? 0x18 : 0;
+    tp.mask = (dl % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
-    for (int t = 0; t < p->desc.m; ++t) {
-        tp.nb_div[t] = make_fast_div((int)p->desc.st[t].nblocks);
-        tp.s_div[t] = make_fast_div((int)p->desc.st[t].s);
+    tp.last_blocks = p->d_blocks + pd.st[pd.m - 1].block_off;
+    for (int t = 0; t < pd.m; ++t) {
+        tp.nb_div[t] = make_fast_div((int)(dl / pd.st[t].b));
+        tp.s_div[t] = make_fast_div((int)pd.st[t].s);
         if (!fast_div_ok(tp.nb_div[t]) || !fast_div_ok(tp.s_div[t])) return HARP_ERR_UNSUPPORTED;
     }
-    const size_t smem = (size_t)R * d * 4 + (size_t)staged * d * es_in + 16;
-    const int grid = (int)std::min<int64_t>(tp.ntiles, sm_count());
+    const size_t smem = (size_t)R * dl * 4 + (size_t)staged * dl * es_in + 16;
+    const int grid = cl * (int)std::min<int64_t>(tp.ntiles, sm_count() / cl);
     int nt = kThreadChoices[1];
     {
         const int qv = (int)((std::min<int64_t>(R, rows) + V - 1) / V);
-        for (int t = 0; t < p->desc.m; ++t)
-            if (stage_groups((int)p->desc.st[t].nblocks, qv, kThreadChoices[1]) > 1) nt = kThreadChoices[0];
+        for (int t = 0; t < pd.m - (cl == 2 ? 1 : 0); ++t)
+            if (stage_groups((int)(dl / pd.st[t].b), qv, kThreadChoices[1]) > 1) nt = kThreadChoices[0];
     }
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;
     cudaError_t e;
     if (in_dtype == HARP_BF16 && out_dtype == HARP_BF16)
-        e = harp_tiled_launch_bf16(which, V, nt, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16(which, V, nt, cl, inv, tp, smem, grid, s);
     else if (in_dtype == HARP_F32)
-        e = harp_tiled_launch_f32(which, V, nt, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_f32(which, V, nt, cl, inv, tp, smem, grid, s);
     else
-        e = harp_tiled_launch_bf16_f32(which, V, nt, inv, tp, smem, grid, s);
+        e = harp_tiled_launch_bf16_f32(which, V, nt, cl, inv, tp, smem, grid, s);
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_tiled_kernel");
     return HARP_OK;

@@ -63,8 +63,9 @@ struct TiledParams {
     int staged_rows;            // the first rows of the next tile that arrive by bulk copy
     int mask;                   // V = 1 swizzle: 0x18 when d % 32 == 0, else 0
     int* status;
-    FastDiv nb_div[HARP_MAX_STAGES];   // division by d / b_t
+    FastDiv nb_div[HARP_MAX_STAGES];   // division by (coordinates per CTA) / b_t
     FastDiv s_div[HARP_MAX_STAGES];    // division by s_t
+    const float* last_blocks;          // slab mode: plain 2 x 2 blocks of the last stage
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -110,6 +111,40 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Both CTAs of the cluster reach this point; shared-memory writes before it are
+// visible to the partner after it.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_cluster4(uint32_t addr, const float4& v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
 }
 
 // ------------------------------------------------------------ helpers ---
@@ -276,16 +311,49 @@ __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, c
     }
 }
 
+// The first staged_rows rows of a tile, columns [col0, col0 + dl), to the staging area.
 template <typename TIn>
-__device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, unsigned char* stage_buf,
-                                           uint64_t* bar) {
-    const int d = (int)p.pd.d;
+__device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, int dl, int col0,
+                                           unsigned char* stage_buf, uint64_t* bar) {
     const int64_t row0 = tile * p.R;
     const int nr = (int)min((int64_t)p.staged_rows, p.rows - row0);
-    const uint32_t row_bytes = (uint32_t)d * sizeof(TIn);
+    const uint32_t row_bytes = (uint32_t)dl * sizeof(TIn);
     mbar_arrive_expect_tx(bar, row_bytes * nr);
-    const TIn* x = (const TIn*)p.x;
+    const TIn* x = (const TIn*)p.x + col0;
     for (int r = 0; r < nr; ++r) bulk_load(stage_buf + (size_t)r * row_bytes, x + (row0 + r) * p.ld_x, row_bytes, bar);
+}
+
+// Slab mode, the last stage (radix 2, stride dl = d / 2): position p of the two slabs
+// forms a group; this CTA (cluster rank r) computes positions p in [r dl/2, (r+1) dl/2)
+// for both slabs, reading and writing the partner's quads through distributed shared
+// memory.  Block c = p; each output sums over its two inputs in order.
+template <bool INV, int NT>
+__device__ __forceinline__ void cross_stage(float4* tile, int dl, int qv, uint32_t rank,
+                                            const float* __restrict__ blocks) {
+    const int half = dl / 2;
+    for (int q = 0; q < qv; ++q) {
+        float4* st = tile + q * dl;
+        for (int pp = threadIdx.x; pp < half; pp += NT) {
+            const int pos = (int)rank * half + pp;
+            float4* own = st + slot<4>(pos, 0);
+            const uint32_t rem = map_to_rank((uint32_t)__cvta_generic_to_shared(own), rank ^ 1);
+            const float4 a = *own, b = ld_cluster4(rem);
+            const float4 x0 = rank == 0 ? a : b, x1 = rank == 0 ? b : a;   // slab 0, slab 1
+            const float4 w = __ldg((const float4*)blocks + pos);          // B[0][0], B[0][1], B[1][0], B[1][1]
+            const float w00 = w.x, w01 = INV ? w.z : w.y, w10 = INV ? w.y : w.z, w11 = w.w;
+            float4 y0, y1;
+            y0.x = fmaf(w01, x1.x, fmaf(w00, x0.x, 0.f));
+            y0.y = fmaf(w01, x1.y, fmaf(w00, x0.y, 0.f));
+            y0.z = fmaf(w01, x1.z, fmaf(w00, x0.z, 0.f));
+            y0.w = fmaf(w01, x1.w, fmaf(w00, x0.w, 0.f));
+            y1.x = fmaf(w11, x1.x, fmaf(w10, x0.x, 0.f));
+            y1.y = fmaf(w11, x1.y, fmaf(w10, x0.y, 0.f));
+            y1.z = fmaf(w11, x1.z, fmaf(w10, x0.z, 0.f));
+            y1.w = fmaf(w11, x1.w, fmaf(w10, x0.w, 0.f));
+            *own = rank == 0 ? y0 : y1;
+            st_cluster4(rem, rank == 0 ? y1 : y0);
+        }
+    }
 }
 
 // Rows -> sub-tiles.  V = 4: a thread takes 8 consecutive coordinates of the 4 rows of a
@@ -374,7 +442,10 @@ __device__ __forceinline__ void drain_tile(const typename VecOf<V>::T* tile, int
     }
 }
 
-template <typename TIn, typename TOut, bool INV, int MASK, int V, int NT>
+// CL = 1: one CTA holds whole rows.  CL = 2 (slab mode, schedules whose last radix is 2):
+// a cluster of two CTAs shares each tile, CTA r holding columns [r d/2, (r+1) d/2) of its
+// rows; stages 0..m-2 stay inside a slab, the last one is cross_stage.
+template <typename TIn, typename TOut, bool INV, int MASK, int V, int NT, int CL>
 __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant__ TiledParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     using VT = typename VecOf<V>::T;
@@ -382,51 +453,35 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
     const int m = p.pd.m;
     const int R = p.R;
     const int tid = threadIdx.x;
+    const uint32_t rank = CL == 2 ? cluster_rank() : 0;
+    const int dl = d / CL;                  // coordinates of a row held by this CTA
+    const int col0 = (int)rank * dl;
+    const int m_local = CL == 2 ? m - 1 : m;
     VT* tile = (VT*)smem;
-    unsigned char* stage_buf = smem + (size_t)R * d * sizeof(float);
-    uint64_t* bar = (uint64_t*)(stage_buf + (size_t)p.staged_rows * d * sizeof(TIn));
+    unsigned char* stage_buf = smem + (size_t)R * dl * sizeof(float);
+    uint64_t* bar = (uint64_t*)(stage_buf + (size_t)p.staged_rows * dl * sizeof(TIn));
 
-    int64_t t_idx = blockIdx.x;
-    if (t_idx >= p.ntiles) return;
+    int64_t t_idx = blockIdx.x / CL;
+    const int64_t t_step = gridDim.x / CL;
+    if (t_idx >= p.ntiles) return;          // both CTAs of a cluster have the same t_idx
     if (p.staged_rows) {
         if (tid == 0) mbar_init(bar, 1);
         __syncthreads();
-        if (tid == 0) issue_tile<TIn>(p, t_idx, stage_buf, bar);
+        if (tid == 0) issue_tile<TIn>(p, t_idx, dl, col0, stage_buf, bar);
     }
-    // The stage order: forward 0..m-1, inverse m-1..0.
-    auto stage_of = [&](int step) { return INV ? m - 1 - step : step; };
-    uint32_t parity = 0;
-    for (; t_idx < p.ntiles; t_idx += gridDim.x) {
-        const int64_t row0 = t_idx * R;
-        const int nr = (int)min((int64_t)R, p.rows - row0);
-        const int qv = (nr + V - 1) / V;
-        const int n_staged = min(nr, p.staged_rows);
-        if (n_staged) {
-            const bool ok = mbar_wait(bar, parity);
-            parity ^= 1;
-            if (__syncthreads_or(!ok)) {
-                if (tid == 0) atomicExch(p.status, 1);
-                return;
-            }
-        }
-        fill_tile<V, NT, TIn>(tile, d, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x, p.ld_x,
-                          p.mask);
-        __syncthreads();
-        const int64_t t_next = t_idx + gridDim.x;
-        if (p.staged_rows && tid == 0 && t_next < p.ntiles) {
-            fence_proxy_async_smem();   // the staging reads above happen before the copies' writes
-            issue_tile<TIn>(p, t_next, stage_buf, bar);
-        }
-        for (int step = 0; step < m; ++step) {
-            const int t = stage_of(step);
+    // local stages in order: forward 0..m_local-1, inverse m_local-1..0
+    auto local_stages = [&](int qv) {
+        for (int step = 0; step < m_local; ++step) {
+            const int t = INV ? m_local - 1 - step : step;
             const StageDesc& sd = p.pd.st[t];
-            const float* sb = p.lanes + p.lane_off[t];
+            // the slab's blocks of stage t start at block r dl / b_t
+            const float* sb = p.lanes + p.lane_off[t] + (int64_t)rank * dl * sd.b;
             const int s = (int)sd.s;
             switch (sd.b) {
-#define HARP_TILED_CASE(R)                                                                          \
-    case R:                                                                                         \
-        if constexpr ((MASK >> R) & 1)                                                              \
-            run_stage<R, INV, V, NT>(sb, s, p.nb_div[t], p.s_div[t], tile, d, qv, p.mask);          \
+#define HARP_TILED_CASE(RB)                                                                         \
+    case RB:                                                                                        \
+        if constexpr ((MASK >> RB) & 1)                                                             \
+            run_stage<RB, INV, V, NT>(sb, s, p.nb_div[t], p.s_div[t], tile, dl, qv, p.mask);       \
         break;
                 HARP_TILED_CASE(2) HARP_TILED_CASE(3) HARP_TILED_CASE(4) HARP_TILED_CASE(5)
                 HARP_TILED_CASE(6) HARP_TILED_CASE(7) HARP_TILED_CASE(8)
@@ -435,7 +490,40 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
             }
             __syncthreads();
         }
-        drain_tile<V, NT, TOut>(tile, d, nr, (TOut*)p.y + row0 * p.ld_y, p.ld_y, p.mask);
+    };
+    uint32_t parity = 0;
+    bool failed = false;    // a bounded wait gave up: keep every barrier, skip the waits
+    for (; t_idx < p.ntiles; t_idx += t_step) {
+        const int64_t row0 = t_idx * R;
+        const int nr = (int)min((int64_t)R, p.rows - row0);
+        const int qv = (nr + V - 1) / V;
+        const int n_staged = min(nr, p.staged_rows);
+        if (n_staged && !failed) {
+            const bool ok = mbar_wait(bar, parity);
+            parity ^= 1;
+            if (__syncthreads_or(!ok)) {
+                if (tid == 0) atomicExch(p.status, 1);
+                failed = true;
+            }
+        }
+        fill_tile<V, NT, TIn>(tile, dl, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x + col0,
+                              p.ld_x, p.mask);
+        __syncthreads();
+        const int64_t t_next = t_idx + t_step;
+        if (p.staged_rows && tid == 0 && t_next < p.ntiles && !failed) {
+            fence_proxy_async_smem();   // the staging reads above happen before the copies' writes
+            issue_tile<TIn>(p, t_next, dl, col0, stage_buf, bar);
+        }
+        if constexpr (CL == 2) {
+            if (!INV) local_stages(qv);
+            cluster_sync();             // both slabs of the tile are ready
+            cross_stage<INV, NT>((float4*)tile, dl, qv, rank, p.last_blocks);
+            cluster_sync();             // the partner's writes into this tile are visible
+            if (INV) local_stages(qv);
+        } else {
+            local_stages(qv);
+        }
+        drain_tile<V, NT, TOut>(tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0, p.ld_y, p.mask);
         __syncthreads();
     }
 }
@@ -455,17 +543,38 @@ constexpr bool has_row_major_kernel(int mask) { return ((mask >> 5) & 1) == 0; }
 // over them without dividing the tile's sub-tiles between items; else 256.
 constexpr int kThreadChoices[] = {256, 384};
 
-template <typename TIn, typename TOut, bool INV, int V, int NT, int I>
+// Slab-mode kernels exist for the radix sets that contain 2.
+constexpr bool has_slab_kernel(int mask) { return ((mask >> 2) & 1) != 0 && mask != 0x1fc; }
+
+template <typename TIn, typename TOut, bool INV, int V, int NT, int CL, int I>
 cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
     if constexpr (I < kNumMasks) {
-        if (which != I) return launch_mask<TIn, TOut, INV, V, NT, I + 1>(which, tp, smem, grid, stream);
-        if constexpr (V == 1 && !has_row_major_kernel(kMasks[I])) {
+        if (which != I) return launch_mask<TIn, TOut, INV, V, NT, CL, I + 1>(which, tp, smem, grid, stream);
+        if constexpr ((V == 1 && !has_row_major_kernel(kMasks[I])) ||
+                      (CL == 2 && (V != 4 || !has_slab_kernel(kMasks[I])))) {
             return cudaErrorInvalidValue;
         } else {
-            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT>;
+            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT, CL>;
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
-            kern<<<(unsigned)grid, NT, smem, stream>>>(tp);
+            if constexpr (CL == 1) {
+                kern<<<(unsigned)grid, NT, smem, stream>>>(tp);
+            } else {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3((unsigned)grid);
+                cfg.blockDim = dim3(NT);
+                cfg.dynamicSmemBytes = smem;
+                cfg.stream = stream;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = 2;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                e = cudaLaunchKernelEx(&cfg, kern, tp);
+                if (e != cudaSuccess) return e;
+            }
             return cudaGetLastError();
         }
     } else {
@@ -474,27 +583,31 @@ cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid,
 }
 
 template <typename TIn, typename TOut, bool INV, int V>
-cudaError_t launch_nt(int which, int nt, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
-    if (nt == 384) return launch_mask<TIn, TOut, INV, V, 384, 0>(which, tp, smem, grid, stream);
-    return launch_mask<TIn, TOut, INV, V, 256, 0>(which, tp, smem, grid, stream);
+cudaError_t launch_nt(int which, int nt, int cl, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
+    if (cl == 2) {
+        if (nt == 384) return launch_mask<TIn, TOut, INV, V, 384, 2, 0>(which, tp, smem, grid, stream);
+        return launch_mask<TIn, TOut, INV, V, 256, 2, 0>(which, tp, smem, grid, stream);
+    }
+    if (nt == 384) return launch_mask<TIn, TOut, INV, V, 384, 1, 0>(which, tp, smem, grid, stream);
+    return launch_mask<TIn, TOut, INV, V, 256, 1, 0>(which, tp, smem, grid, stream);
 }
 
 template <typename TIn, typename TOut>
-cudaError_t launch(int which, int V, int nt, bool inverse, const TiledParams& tp, size_t smem, int grid,
+cudaError_t launch(int which, int V, int nt, int cl, bool inverse, const TiledParams& tp, size_t smem, int grid,
                    cudaStream_t stream) {
     if (V == 4)
-        return inverse ? launch_nt<TIn, TOut, true, 4>(which, nt, tp, smem, grid, stream)
-                       : launch_nt<TIn, TOut, false, 4>(which, nt, tp, smem, grid, stream);
-    return inverse ? launch_nt<TIn, TOut, true, 1>(which, nt, tp, smem, grid, stream)
-                   : launch_nt<TIn, TOut, false, 1>(which, nt, tp, smem, grid, stream);
+        return inverse ? launch_nt<TIn, TOut, true, 4>(which, nt, cl, tp, smem, grid, stream)
+                       : launch_nt<TIn, TOut, false, 4>(which, nt, cl, tp, smem, grid, stream);
+    return inverse ? launch_nt<TIn, TOut, true, 1>(which, nt, cl, tp, smem, grid, stream)
+                   : launch_nt<TIn, TOut, false, 1>(which, nt, cl, tp, smem, grid, stream);
 }
 
 }  // namespace harp_tiled
 
 // One translation unit per I/O type pair (compiled in parallel).
-cudaError_t harp_tiled_launch_bf16(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_bf16(int which, int V, int nt, int cl, bool inverse, const harp_tiled::TiledParams& tp,
                                    size_t smem, int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_f32(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_f32(int which, int V, int nt, int cl, bool inverse, const harp_tiled::TiledParams& tp,
                                   size_t smem, int grid, cudaStream_t stream);
-cudaError_t harp_tiled_launch_bf16_f32(int which, int V, int nt, bool inverse, const harp_tiled::TiledParams& tp,
+cudaError_t harp_tiled_launch_bf16_f32(int which, int V, int nt, int cl, bool inverse, const harp_tiled::TiledParams& tp,
                                        size_t smem, int grid, cudaStream_t stream);

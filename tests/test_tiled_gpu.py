@@ -134,3 +134,22 @@ def test_default_dispatch_takes_the_tiled_kernel_for_c3_and_c5(monkeypatch):
         run(gp, W.draw_encoded(W.get(name), 0, 64), direction)
         assert H.last_kernel() == "harp_tiled_kernel", name
         gp.device_status()
+
+
+@pytest.mark.parametrize("name", ["c3", "c5"])
+@pytest.mark.parametrize("direction", ["forward", "inverse"])
+def test_slab_mode_matches_whole_rows(monkeypatch, name, direction):
+    """Slab mode (HARP_TILED_SLAB=1): schedules ending in radix 2 at large d run as CTA pairs
+    that each hold half of every row (the last stage exchanged through distributed shared
+    memory); the result is the same, bit for bit, as whole rows in one CTA, and matches the
+    oracle."""
+    gp, tr = plans(name)
+    enc = W.draw_encoded(W.get(name), 0, 301)
+    monkeypatch.setenv("HARP_KERNEL", "tiled")
+    monkeypatch.setenv("HARP_TILED_SLAB", "1")
+    a = run(gp, enc, direction)
+    monkeypatch.setenv("HARP_TILED_SLAB", "0")
+    b = run(gp, enc, direction)
+    np.testing.assert_array_equal(a, b)
+    check(a, tr.apply(decode(enc), direction), decode(enc), f"slab {name} {direction}")
+    gp.device_status()
