@@ -390,7 +390,7 @@ def side_measurements(args, H, W, torch, device, peak):
     ms = e0.elapsed_time(e1) / st
     b4 = 2 * (2 * w4.n_out * w4.n_in * 2)        # two passes, each reading and writing W once
     out.append({"workload": WORKLOAD_TEXT["c4"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
-                "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided (4 launches)"})
+                "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
     del wt, wo, ws
     return out
 
