@@ -131,11 +131,40 @@ HARP_API harp_status harp_materialize_blocks(harp_plan_t plan, void* stream);
  *   rows        number of rows; 0 is a no-op returning HARP_OK.
  *   ld_x, ld_y  leading dimensions in elements, >= d.
  * Arithmetic: inputs widened to fp32, every stage accumulated in fp32 with fused
- * multiply-adds, the output rounded to `dtype` to nearest even.
+ * multiply-adds (the specialized d = 4096 kernel forms the products on tensor cores from
+ * TF32 hi/lo splits of both operands, three passes, fp32 accumulation), the output
+ * rounded to `dtype` to nearest even.
  */
 HARP_API harp_status harp_apply(harp_plan_t plan, const void* x, void* y, int64_t rows,
                        int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
                        void* stream);
+
+/*
+ * harp_apply_ex — harp_apply with separate input and output types (for example bf16 rows
+ * in, fp32 rows out, to keep an intermediate unrounded).  y may equal x only when the two
+ * types are equal.  Everything else as harp_apply.
+ */
+HARP_API harp_status harp_apply_ex(harp_plan_t plan, const void* x, void* y, int64_t rows,
+                                   int64_t ld_x, int64_t ld_y, harp_dtype in_dtype,
+                                   harp_dtype out_dtype, harp_dir dir, void* stream);
+
+/*
+ * harp_apply_columns — every column of an fp32 matrix takes T (FORWARD) or T^T
+ * (INVERSE): for j < ncols, y[:, j] = T x[:, j] with x of d = plan dimension rows.  The
+ * column side of a two-sided rotation, applied in place without a transpose (HARP
+ * abstract: a rotation on each side of a weight matrix).
+ *   x        device fp32 matrix, d rows of ncols, leading dimension ld_x >= ncols,
+ *            16-byte aligned, ld_x a multiple of 4.  Overwritten (it holds an
+ *            intermediate between the kernel's two passes).
+ *   y        result, d rows of ncols, leading dimension ld_y (a multiple of 4 elements),
+ *            16-byte aligned, element type out_dtype; y may equal x for HARP_F32.
+ * Returns HARP_ERR_UNSUPPORTED for plans the column kernel does not take (a single
+ * stage, a radix above 8, a schedule without a split whose tiles fit in shared memory)
+ * and for unaligned arguments.
+ */
+HARP_API harp_status harp_apply_columns(harp_plan_t plan, float* x, int64_t ld_x, int64_t ncols,
+                                        void* y, int64_t ld_y, harp_dtype out_dtype, harp_dir dir,
+                                        void* stream);
 
 /*
  * harp_two_sided_workspace_bytes — device workspace that harp_apply_two_sided

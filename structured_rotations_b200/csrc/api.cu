@@ -64,12 +64,14 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 }  // namespace
 
-extern "C" harp_status harp_apply(harp_plan_t p, const void* x, void* y, int64_t rows,
-                                  int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
-                                  void* stream) {
+namespace {
+
+harp_status apply_checked(harp_plan_t p, const void* x, void* y, int64_t rows, int64_t ld_x, int64_t ld_y,
+                          harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir, void* stream) {
     harp_clear_error();
     if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
-    if (dtype != HARP_F32 && dtype != HARP_BF16) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown dtype");
+    if ((in_dtype != HARP_F32 && in_dtype != HARP_BF16) || (out_dtype != HARP_F32 && out_dtype != HARP_BF16))
+        return harp_fail(HARP_ERR_UNSUPPORTED, "unknown dtype");
     if (dir != HARP_FORWARD && dir != HARP_INVERSE) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown direction");
     if (rows < 0) return harp_fail(HARP_ERR_INVALID_ARG, "rows < 0");
     const int64_t d = p->desc.d;
@@ -79,13 +81,54 @@ extern "C" harp_status harp_apply(harp_plan_t p, const void* x, void* y, int64_t
     if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
     harp_status st = check_device(p);
     if (st != HARP_OK) return st;
-    const size_t es = esize(dtype);
+    const size_t es_in = esize(in_dtype), es_out = esize(out_dtype);
     if (x == y) {
-        if (ld_x != ld_y) return harp_fail(HARP_ERR_INVALID_ARG, "in-place apply needs ld_x == ld_y");
-    } else if (ranges_overlap(x, ((rows - 1) * ld_x + d) * es, y, ((rows - 1) * ld_y + d) * es)) {
+        if (ld_x != ld_y || in_dtype != out_dtype)
+            return harp_fail(HARP_ERR_INVALID_ARG, "in-place apply needs ld_x == ld_y and one element type");
+    } else if (ranges_overlap(x, ((rows - 1) * ld_x + d) * es_in, y, ((rows - 1) * ld_y + d) * es_out)) {
         return harp_fail(HARP_ERR_INVALID_ARG, "x and y overlap without being equal");
     }
-    return run_rows(p, x, y, rows, ld_x, ld_y, dtype, dtype, dir, stream);
+    return run_rows(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
+}
+
+}  // namespace
+
+extern "C" harp_status harp_apply(harp_plan_t p, const void* x, void* y, int64_t rows,
+                                  int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
+                                  void* stream) {
+    return apply_checked(p, x, y, rows, ld_x, ld_y, dtype, dtype, dir, stream);
+}
+
+extern "C" harp_status harp_apply_ex(harp_plan_t p, const void* x, void* y, int64_t rows, int64_t ld_x,
+                                     int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
+                                     void* stream) {
+    return apply_checked(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
+}
+
+extern "C" harp_status harp_apply_columns(harp_plan_t p, float* x, int64_t ld_x, int64_t ncols, void* y,
+                                          int64_t ld_y, harp_dtype out_dtype, harp_dir dir, void* stream) {
+    harp_clear_error();
+    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    if (out_dtype != HARP_F32 && out_dtype != HARP_BF16) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown dtype");
+    if (dir != HARP_FORWARD && dir != HARP_INVERSE) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown direction");
+    if (ncols < 0) return harp_fail(HARP_ERR_INVALID_ARG, "ncols < 0");
+    if (ld_x < ncols || ld_y < ncols) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than ncols");
+    if (ncols == 0) return HARP_OK;
+    if (!x || !y) return harp_fail(HARP_ERR_INVALID_ARG, "x or y is NULL");
+    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    harp_status st = check_device(p);
+    if (st != HARP_OK) return st;
+    const int64_t d = p->desc.d;
+    const size_t xb = ((d - 1) * ld_x + ncols) * sizeof(float), yb = ((d - 1) * ld_y + ncols) * esize(out_dtype);
+    if ((void*)x == y) {
+        if (ld_x != ld_y || out_dtype != HARP_F32)
+            return harp_fail(HARP_ERR_INVALID_ARG, "in place needs ld_x == ld_y and fp32 output");
+    } else if (ranges_overlap(x, xb, y, yb)) {
+        return harp_fail(HARP_ERR_INVALID_ARG, "x and y overlap without being equal");
+    }
+    st = launch_cols(p, x, ld_x, ncols, y, ld_y, out_dtype, dir, stream);
+    if (st == HARP_ERR_UNSUPPORTED) return harp_fail(st, "shape or alignment not covered by the column kernel");
+    return st;
 }
 
 extern "C" size_t harp_two_sided_workspace_bytes(int64_t n_out, int64_t n_in) {

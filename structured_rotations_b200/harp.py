@@ -63,6 +63,8 @@ def lib():
                                       _c_i32, _vp, ctypes.POINTER(ctypes.c_float), _c_u64, _c_u64]),
         "harp_materialize_blocks": (_c_i32, [_vp, _vp]),
         "harp_apply": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32, _vp]),
+        "harp_apply_ex": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32, _c_i32, _vp]),
+        "harp_apply_columns": (_c_i32, [_vp, _vp, _c_i64, _c_i64, _vp, _c_i64, _c_i32, _c_i32, _vp]),
         "harp_two_sided_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64]),
         "harp_apply_two_sided": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp,
                                           ctypes.c_size_t, _vp]),
@@ -190,6 +192,32 @@ class Plan:
         d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
         _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
                                 _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
+        return y
+
+    def apply_ex(self, x, y, direction: str = "forward", stream=None):
+        """Rows of x (float32 or bfloat16) into y of its own type (harp_apply_ex), e.g. bf16
+        rows into an fp32 intermediate."""
+        if x.shape[-1] != self.d or y.shape[-1] != self.d or x.shape[0] != y.shape[0]:
+            raise ValueError(f"x and y must both be rows of d={self.d}")
+        d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
+        _check(lib().harp_apply_ex(self._h, x.data_ptr(), y.data_ptr(), x.shape[0], _ld(x), _ld(y),
+                                   _dtype_code(x), _dtype_code(y), d, _stream_handle(stream)), "harp_apply_ex")
+        return y
+
+    def apply_columns(self, x, y=None, direction: str = "forward", stream=None):
+        """Every column of the fp32 matrix x (d rows) takes T or T^T (harp_apply_columns);
+        y defaults to x itself (in place); a bfloat16 y receives the rounded result.  x is
+        overwritten either way."""
+        import torch
+        if x.dtype != torch.float32 or x.shape[0] != self.d:
+            raise ValueError(f"x must be float32 with d={self.d} rows")
+        if y is None:
+            y = x
+        if y.shape != x.shape:
+            raise ValueError("y must have the shape of x")
+        d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
+        _check(lib().harp_apply_columns(self._h, x.data_ptr(), _ld(x), x.shape[1], y.data_ptr(), _ld(y),
+                                        _dtype_code(y), d, _stream_handle(stream)), "harp_apply_columns")
         return y
 
     def device_status(self) -> None:

@@ -105,3 +105,52 @@ def test_bench_reference_arm_under_torchrun_prints_once():
     out = json.loads(lines[0])
     assert out["impl"] == "reference" and out["value"] > 0 and out["n_gpus"] == 2
     assert out["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _two_sided_worker(rank, world, port, out_dir):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import workloads as W
+    from oracle import harp_oracle as O
+    from structured_rotations_b200.shard import two_sided_row_sharded
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        u_s, v_s = (8, 2, 4), (4, 2, 2)                       # n_out 64, n_in 16
+        tu = O.Transform(O.make_plan(64, u_s, W.draw_theta(O.theta_count(u_s), 0.3, 5), sign_seed=6))
+        tv = O.Transform(O.make_plan(16, v_s, W.draw_theta(O.theta_count(v_s), 0.3, 7), sign_seed=8))
+        w = np.random.default_rng(11).standard_normal((64, 16))
+        n = 64 // world
+        w_local = torch.from_numpy(w[rank * n:(rank + 1) * n].copy())
+
+        def row_fn(src, dst):
+            dst.copy_(torch.from_numpy(tv.inverse(src.numpy())))
+
+        def col_fn(src, dst):
+            dst.copy_(torch.from_numpy(tu.inverse(src.numpy().T).T))
+
+        out = two_sided_row_sharded(None, None, w_local, work_dtype=torch.float64, row_fn=row_fn, col_fn=col_fn)
+        parts = [None] * world
+        dist.all_gather_object(parts, out.numpy())
+        if rank == 0:
+            got = np.concatenate(parts)
+            want = tu.inverse(tv.inverse(w).T).T                 # T_U^T W T_V
+            with open(os.path.join(out_dir, "two_sided.json"), "w") as f:
+                json.dump({"max_err": float(np.abs(got - want).max()), "shape": list(got.shape)}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_two_sided_row_sharded_exchange(tmp_path, world):
+    """The row-sharded two-sided rotation (rows local, all-to-all, columns local,
+    all-to-all back) on gloo ranks, with a float64 reference as each rank's compute,
+    equals the single-process T_U^T W T_V."""
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.spawn(_two_sided_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    r = json.load(open(tmp_path / "two_sided.json"))
+    assert r["shape"] == [64, 16]
+    assert r["max_err"] < 1e-12

@@ -93,3 +93,49 @@ def test_unaligned_columns_fall_back(monkeypatch):
     assert H.last_kernel() != "harp_cols_kernel"
     want = tu.inverse(tv.inverse(w.astype(np.float32).astype(np.float64)).T).T
     check_f32(out, want, np.full(pu.d, np.max(np.linalg.norm(enc.astype(np.float64), axis=1))), "fallback")
+
+
+@pytest.mark.parametrize("sched", [(8, 8, 8, 7), (8, 8, 2), (5, 2, 8), (2, 8, 8)])
+@pytest.mark.parametrize("direction", ["forward", "inverse"])
+@pytest.mark.parametrize("out", ["f32", "bf16", "in_place"])
+def test_apply_columns_vs_oracle(sched, direction, out):
+    gp, tr = _pair(sched, 91)
+    d, ncols = gp.d, 200
+    x = np.random.default_rng(d + ncols).standard_normal((d, ncols)).astype(np.float32)
+    xt = to_dev(x)
+    if out == "in_place":
+        y = gp.apply_columns(xt, direction=direction)
+    else:
+        yt = torch.empty(d, ncols, device=xt.device, dtype=torch.bfloat16 if out == "bf16" else torch.float32)
+        y = gp.apply_columns(xt, yt, direction=direction)
+    torch.cuda.synchronize()
+    assert H.last_kernel() == "harp_cols_kernel"
+    want = tr.apply(x.astype(np.float64).T, direction).T          # every column
+    got = to_host(y)
+    cn = np.linalg.norm(x.astype(np.float64), axis=0)              # column norms
+    if out == "bf16":
+        check_bf16(got.T.copy(), want.T, cn, O.round_bf16, f"columns {sched} {direction}")
+    else:
+        check_f32(got.T, want.T, cn, f"columns {sched} {direction}")
+
+
+def test_apply_ex_bf16_rows_to_f32():
+    gp, tr = _pair((8, 8, 8, 8, 2), 93)
+    enc = W.encode_bf16(np.random.default_rng(5).standard_normal((70, gp.d)))
+    x = to_dev(enc)
+    y = torch.empty(70, gp.d, device=x.device, dtype=torch.float32)
+    gp.apply_ex(x, y, direction="inverse")
+    torch.cuda.synchronize()
+    xf = decode(enc)
+    check_f32(to_host(y), tr.inverse(xf), np.linalg.norm(xf, axis=1), "apply_ex bf16 -> f32")
+
+
+def test_row_sharded_two_sided_on_one_rank_equals_two_sided():
+    from structured_rotations_b200.shard import two_sided_row_sharded
+    pu, _ = _pair((8, 8, 8, 7), 95)
+    pv, _ = _pair((8, 8, 8, 2), 96)
+    w = to_dev(W.encode_bf16(np.random.default_rng(9).standard_normal((pu.d, pv.d)) * 0.02))
+    a = two_sided_row_sharded(pu, pv, w)
+    b = H.apply_two_sided(pu, pv, w)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
