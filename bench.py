@@ -315,28 +315,26 @@ def time_apply(plan, x, y, steps, warmup, torch, dist=None, direction="forward")
 
 
 def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
+    """The same metric through the public host-buffer call (harp_apply_host): every step
+    copies this rank's rows from pinned host memory to the GPU, rotates them and copies
+    them back, chunk by chunk on overlapping streams; host wall clock around the
+    synchronous call, max over ranks."""
     import numpy as np
     xh = torch.from_numpy(enc.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty_like(xh).pin_memory()
-    stream = torch.cuda.current_stream()
     for _ in range(2):
-        x.copy_(xh, non_blocking=True); plan.apply(x, y); yh.copy_(y, non_blocking=True)
+        plan.apply_host(xh, yh)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    t0 = time.perf_counter()
     for _ in range(args.e2e_steps):
-        x.copy_(xh, non_blocking=True)
-        plan.apply(x, y)
-        yh.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, dist, device)
-    e2e = {"value": world * rows * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+        plan.apply_host(xh, yh)
+    e2e_s = time.perf_counter() - t0
+    e2e_s = max_over_ranks(e2e_s, dist, device)
+    e2e = {"value": world * rows * args.e2e_steps / e2e_s, "unit": UNIT,
            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
-           "path": "pinned host -> device copy, harp_apply, device -> pinned host copy, one stream"}
+           "path": "harp_apply_host: pinned host rows -> GPU -> pinned host rows, 32 MiB chunks on 3 streams"}
     del xh, yh
     return e2e
 

@@ -149,6 +149,21 @@ HARP_API harp_status harp_apply_ex(harp_plan_t plan, const void* x, void* y, int
                                    harp_dtype out_dtype, harp_dir dir, void* stream);
 
 /*
+ * harp_apply_host — harp_apply between host buffers, copies included: y_r = T x_r
+ * (FORWARD) or T^T x_r (INVERSE) for rows in host memory.  The rows pass through the GPU in
+ * chunks of about 32 MiB on three streams owned by the plan, so that host-to-device copies,
+ * kernels and device-to-host copies overlap (page-locked host memory is needed for the
+ * overlap; pageable memory works, the copies then serialize).  Synchronous: returns when y
+ * holds the result.  Runs on the current device, which must be the plan's.  The plan keeps
+ * the streams and six device buffers of one chunk until harp_plan_destroy.
+ *   x, y        host pointers, element type dtype; y may equal x (then ld_x == ld_y); any
+ *               other overlap returns HARP_ERR_INVALID_ARG.
+ *   rows, ld_x, ld_y, dtype, dir   as harp_apply.
+ */
+HARP_API harp_status harp_apply_host(harp_plan_t plan, const void* x, void* y, int64_t rows,
+                                     int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir);
+
+/*
  * harp_apply_columns — every column of an fp32 matrix takes T (FORWARD) or T^T
  * (INVERSE): for j < ncols, y[:, j] = T x[:, j] with x of d = plan dimension rows.  The
  * column side of a two-sided rotation, applied in place without a transpose (HARP

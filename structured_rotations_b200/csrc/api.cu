@@ -38,6 +38,8 @@ int kernel_choice() {
     return kAuto;
 }
 
+}  // namespace
+
 // The row kernels in order of preference.
 harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x, int64_t ld_y,
                      harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir, void* stream) {
@@ -62,7 +64,6 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
     return pa < pb + nb && pb < pa + na;
 }
 
-}  // namespace
 
 namespace {
 

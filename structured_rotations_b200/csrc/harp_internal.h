@@ -55,6 +55,7 @@ struct harp_plan_s {
     int8_t* d_signs = nullptr;
     int* d_status = nullptr;          // device error word (bounded waits)
     void* fast = nullptr;             // fast-path state (see apply_fast.cu)
+    void* host_io = nullptr;          // streams and staging buffers of harp_apply_host (host_io.cu)
 };
 
 // error reporting (plan.cpp)
@@ -79,6 +80,11 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               int64_t ld_x, int64_t ld_y, harp_dtype in_dtype, harp_dir dir,
                               void* stream, harp_dtype out_dtype);
 void fast_state_free(harp_plan_s* p);
+void host_io_free(harp_plan_s* p);
+
+// the row kernels in order of preference (api.cu)
+harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x, int64_t ld_y,
+                     harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir, void* stream);
 
 // Column transform for the two-sided rotation (cols.cu): every column of an fp32 matrix
 // x (d rows) takes T (forward) or T^T (inverse); result to y (fp32, may be x, or bf16).

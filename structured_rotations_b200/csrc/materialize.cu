@@ -121,6 +121,7 @@ harp_status harp_device_free(harp_plan_s* p) {
     cudaSetDevice(p->device);
     cudaDeviceSynchronize();
     fast_state_free(p);
+    host_io_free(p);
     cudaFree(p->d_blocks);
     cudaFree(p->d_blocks_lanes);
     cudaFree(p->d_theta);

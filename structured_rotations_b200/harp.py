@@ -65,6 +65,7 @@ def lib():
         "harp_apply": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32, _vp]),
         "harp_apply_ex": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32, _c_i32, _vp]),
         "harp_apply_columns": (_c_i32, [_vp, _vp, _c_i64, _c_i64, _vp, _c_i64, _c_i32, _c_i32, _vp]),
+        "harp_apply_host": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _c_i32]),
         "harp_two_sided_workspace_bytes": (ctypes.c_size_t, [_c_i64, _c_i64]),
         "harp_apply_two_sided": (_c_i32, [_vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp,
                                           ctypes.c_size_t, _vp]),
@@ -192,6 +193,22 @@ class Plan:
         d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
         _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
                                 _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
+        return y
+
+    def apply_host(self, x, y=None, direction: str = "forward"):
+        """Rows of a host (CPU) tensor through the GPU and back (harp_apply_host): copies,
+        kernels and copies overlap in chunks; pin x and y (tensor.pin_memory()) for the
+        overlap.  Returns y (a new host tensor by default)."""
+        import torch
+        if x.device.type != "cpu":
+            raise ValueError("apply_host takes host tensors; use apply for device tensors")
+        if y is None:
+            y = torch.empty_like(x, pin_memory=x.is_pinned())
+        if x.dtype != y.dtype or x.shape != y.shape or x.shape[-1] != self.d:
+            raise ValueError(f"x and y must be rows of d={self.d} of one dtype")
+        d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
+        _check(lib().harp_apply_host(self._h, x.data_ptr(), y.data_ptr(), x.shape[0], _ld(x), _ld(y),
+                                     _dtype_code(x), d), "harp_apply_host")
         return y
 
     def apply_ex(self, x, y, direction: str = "forward", stream=None):
