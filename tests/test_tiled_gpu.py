@@ -153,3 +153,32 @@ def test_slab_mode_matches_whole_rows(monkeypatch, name, direction):
     np.testing.assert_array_equal(a, b)
     check(a, tr.apply(decode(enc), direction), decode(enc), f"slab {name} {direction}")
     gp.device_status()
+
+
+@pytest.mark.parametrize("schedule", [(8, 8, 8, 8, 8), (8, 8, 8, 8, 7)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_largest_dimensions_single_row_subtiles(tiled, schedule, dtype):
+    """d = 32768 (the largest the library takes) and 28672: fp32 tiles of 4 rows no longer
+    fit in shared memory, so the tiled kernel holds one row per sub-tile."""
+    gp, tr = _plan_pair(schedule, 500 + schedule[-1])
+    d = int(np.prod(schedule))
+    x = np.random.default_rng(d).standard_normal((6, d))
+    enc = W.encode_bf16(x) if dtype == "bf16" else x.astype(np.float32)
+    xf = decode(enc)
+    for direction in ("forward", "inverse"):
+        out = run(gp, enc, direction)
+        check(out, tr.apply(xf, direction), xf, f"d={d} {dtype} {direction}")
+
+
+@pytest.mark.parametrize("schedule", [(2,), (3,), (2, 2), (16,), (16, 3), (12, 5)])
+def test_degenerate_and_large_radix_schedules(monkeypatch, schedule):
+    """One stage, d = 2, radices above 8: the simple kernel takes them."""
+    monkeypatch.delenv("HARP_KERNEL", raising=False)
+    gp, tr = _plan_pair(schedule, 600 + sum(schedule))
+    d = int(np.prod(schedule))
+    x = np.random.default_rng(d + 1).standard_normal((257, d)).astype(np.float32)
+    xf = x.astype(np.float64)
+    for direction in ("forward", "inverse"):
+        out = run(gp, x, direction)
+        check(out, tr.apply(xf, direction), xf, f"{schedule} {direction}")
+    assert H.last_kernel() == "apply_simple_kernel"
