@@ -33,12 +33,12 @@ METRIC = "HARP rotation rows/s and HBM GB/s (fraction of B200 roofline), d=4096/
 UNIT = "rows/s"
 FALLBACK_HBM_GBS = 6650.0
 WORKLOAD_TEXT = {
-    "c2": "d=4096 schedule (8,8,8,8), 65536 rows/GPU bf16 Student-t(3) with 8 outlier channels x50, "
+    "d4096": "d=4096 schedule (8,8,8,8), 65536 rows/GPU bf16 Student-t(3) with 8 outlier channels x50, "
           "theta~N(0,0.05), forward",
-    "c3_64k": "d=5120 schedule (8,8,8,5,2), 65536 rows/GPU bf16 N(0,1) with 1% entries x20, forward",
-    "c4": "two-sided T_U^T W T_V: W 28672x8192 bf16 N(0,0.02^2) with 16 outlier columns x30, "
+    "d5120_64k": "d=5120 schedule (8,8,8,5,2), 65536 rows/GPU bf16 N(0,1) with 1% entries x20, forward",
+    "two_sided": "two-sided T_U^T W T_V: W 28672x8192 bf16 N(0,0.02^2) with 16 outlier columns x30, "
           "U (8,8,8,8,7), V (8,8,8,8,2), theta~N(0,0.05)",
-    "c5": "d=8192 schedule (8,8,8,8,2), int8 theta + per-stage scale, 65536 rows/GPU bf16 N(0,1), forward",
+    "d8192_int8": "d=8192 schedule (8,8,8,8,2), int8 theta + per-stage scale, 65536 rows/GPU bf16 N(0,1), forward",
 }
 
 
@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2", choices=["c2", "c3_64k", "c5"])
+    ap.add_argument("--workload", default="d4096", choices=["d4096", "d5120_64k", "d8192_int8"])
     ap.add_argument("--no-extra", action="store_true", help="skip the d=5120 / d=8192 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -339,8 +339,8 @@ def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
     return e2e
 
 
-SIDE = (("c2", "inverse"), ("c3_64k", "forward"), ("c3_64k", "inverse"), ("c5", "forward"),
-        ("c5", "inverse"))
+SIDE = (("d4096", "inverse"), ("d5120_64k", "forward"), ("d5120_64k", "inverse"), ("d8192_int8", "forward"),
+        ("d8192_int8", "inverse"))
 
 
 def side_measurements(args, H, W, torch, device, peak):
@@ -366,7 +366,7 @@ def side_measurements(args, H, W, torch, device, peak):
         del y2
     cache.clear()
     # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)
-    w4 = W.get("c4")
+    w4 = W.get("two_sided")
     th_v = W.draw_theta(H.theta_count(w4.schedule), w4.theta_sigma, w4.theta_seed)
     th_u = W.draw_theta(H.theta_count(w4.u_schedule), w4.theta_sigma, w4.theta_seed + 7)
     pv = H.Plan(w4.n_in, w4.schedule, theta=th_v, sign_seed=w4.sign_seed).materialize()
@@ -387,7 +387,7 @@ def side_measurements(args, H, W, torch, device, peak):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / st
     b4 = 2 * (2 * w4.n_out * w4.n_in * 2)        # two passes, each reading and writing W once
-    out.append({"workload": WORKLOAD_TEXT["c4"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
+    out.append({"workload": WORKLOAD_TEXT["two_sided"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
                 "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
     del wt, wo, ws
     return out

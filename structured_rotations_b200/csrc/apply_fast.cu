@@ -160,7 +160,7 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* s
         : "memory");
 }
 
-// 2-D tiled TMA load of one box into this CTA's shared memory (no multicast).
+// 2-D tiled TMA load of one box into this CTA's own shared memory.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int col, int row, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"

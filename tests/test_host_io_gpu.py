@@ -26,26 +26,26 @@ def _bits(t):
 
 @pytest.mark.parametrize("direction", ["forward", "inverse"])
 def test_host_chunks_equal_the_device_call(direction):
-    gp, _ = plans("c3")
-    enc = W.draw_encoded(W.get("c3"), 0, 9000)            # three 32 MiB chunks, the last ragged
+    gp, _ = plans("d5120")
+    enc = W.draw_encoded(W.get("d5120"), 0, 9000)            # three 32 MiB chunks, the last ragged
     yh = gp.apply_host(_host(enc), direction=direction)
     yd = gp.apply(to_dev(enc), direction=direction)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(_bits(yh), to_host(yd))
 
 
-def test_host_c2_with_a_small_last_chunk_matches_the_oracle():
-    gp, tr = plans("c2")
-    enc = W.draw_encoded(W.get("c2"), 0, 8200)            # chunks of 4096, 4096 and 8 rows
+def test_host_d4096_with_a_small_last_chunk_matches_the_oracle():
+    gp, tr = plans("d4096")
+    enc = W.draw_encoded(W.get("d4096"), 0, 8200)            # chunks of 4096, 4096 and 8 rows
     out = _bits(gp.apply_host(_host(enc)))
     idx = np.unique(np.concatenate([W.sample_rows(8200, 300), np.arange(8190, 8200)]))
     x = decode(enc[idx])
-    check(out[idx], tr.forward(x), x, "host c2")
+    check(out[idx], tr.forward(x), x, "host d4096")
 
 
 def test_host_in_place_padded_and_pageable():
-    gp, tr = plans("c3")
-    w = W.get("c3")
+    gp, tr = plans("d5120")
+    w = W.get("d5120")
     rows, d, pad = 3100, w.d, 24
     enc = W.draw_encoded(w, 0, rows)
     buf = np.zeros((rows, d + pad), dtype=np.uint16)

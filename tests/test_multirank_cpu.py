@@ -61,7 +61,7 @@ def _worker(rank, world, port, out_dir):
                             timeout=datetime.timedelta(seconds=60))
     try:
         res = {"max": max_over_ranks(10.0 + rank, dist), "max_neg": max_over_ranks(-1.0 - rank, dist)}
-        w = W.get("c3")
+        w = W.get("d5120")
         row0, rows = weak_shard(40, rank)
         enc = W.draw_encoded(w, row0, rows)
         theta = W.draw_theta(O.theta_count(w.schedule), w.theta_sigma, w.theta_seed)

@@ -88,27 +88,27 @@ def run(gp, enc, direction):
 # ---------------------------------------------------------------- workloads ---
 
 @pytest.mark.parametrize("direction", ["forward", "inverse"])
-def test_c1_fp32_full(direction):
-    gp, tr = plans("c1")
-    enc = full_input("c1", 1024)
+def test_d64_fp32_full(direction):
+    gp, tr = plans("d64")
+    enc = full_input("d64", 1024)
     out = run(gp, enc, direction)
-    check(out, tr.apply(decode(enc), direction), decode(enc), f"c1 {direction}")
+    check(out, tr.apply(decode(enc), direction), decode(enc), f"d64 {direction}")
 
 
-def test_c1b_theta_zero_is_randomized_hadamard():
+def test_d64_hadamard_theta_zero_is_randomized_hadamard():
     import scipy.linalg
-    gp, tr = plans("c1b")
-    enc = full_input("c1b", 1024)
+    gp, tr = plans("d64_hadamard")
+    enc = full_input("d64_hadamard", 1024)
     out = run(gp, enc, "forward")
     x = decode(enc)
-    check(out, tr.forward(x), x, "c1b vs oracle")
-    want = (x * O.sign_vector(64, W.get("c1b").sign_seed)) @ scipy.linalg.hadamard(64).T / 8.0
-    check(out, want, x, "c1b vs H_64 S")
+    check(out, tr.forward(x), x, "d64_hadamard vs oracle")
+    want = (x * O.sign_vector(64, W.get("d64_hadamard").sign_seed)) @ scipy.linalg.hadamard(64).T / 8.0
+    check(out, want, x, "d64_hadamard vs H_64 S")
 
 
 @pytest.mark.parametrize("name,direction", [
-    ("c2", "forward"), ("c2", "inverse"), ("c3", "forward"), ("c3", "inverse"),
-    ("c5", "forward"), ("c5", "inverse")])
+    ("d4096", "forward"), ("d4096", "inverse"), ("d5120", "forward"), ("d5120", "inverse"),
+    ("d8192_int8", "forward"), ("d8192_int8", "inverse")])
 @pytest.mark.parametrize("rows", [1, 3, 37, 1000])
 def test_small_batches_full_compare(name, direction, rows):
     gp, tr = plans(name)
@@ -118,11 +118,11 @@ def test_small_batches_full_compare(name, direction, rows):
 
 
 @pytest.mark.parametrize("name,rows,direction", [
-    ("c2", 65536, "forward"),
-    ("c3", 32768, "forward"), ("c3", 32768, "inverse"),
-    ("c3_64k", 65536, "forward"), ("c3_64k", 65536, "inverse"),
-    ("c5", 65536, "forward"), ("c5", 65536, "inverse"),
-    ("c5", 256, "forward"), ("c5", 16, "inverse")])
+    ("d4096", 65536, "forward"),
+    ("d5120", 32768, "forward"), ("d5120", 32768, "inverse"),
+    ("d5120_64k", 65536, "forward"), ("d5120_64k", 65536, "inverse"),
+    ("d8192_int8", 65536, "forward"), ("d8192_int8", 65536, "inverse"),
+    ("d8192_int8", 256, "forward"), ("d8192_int8", 16, "inverse")])
 def test_full_size_sampled(name, rows, direction):
     gp, tr = plans(name)
     enc = full_input(name, rows)
@@ -140,16 +140,16 @@ def test_full_size_sampled(name, rows, direction):
     print(name, direction, rows, stats)
 
 
-def test_c5_decode_rows_one():
-    gp, tr = plans("c5")
-    enc = full_input("c5", 1)
+def test_d8192_int8_decode_rows_one():
+    gp, tr = plans("d8192_int8")
+    enc = full_input("d8192_int8", 1)
     for direction in ("forward", "inverse"):
         out = run(gp, enc, direction)
-        check(out, tr.apply(decode(enc), direction), decode(enc), f"c5 rows=1 {direction}")
+        check(out, tr.apply(decode(enc), direction), decode(enc), f"d8192_int8 rows=1 {direction}")
 
 
 def test_round_trip_fp32_on_device():
-    gp, _ = plans("c3")
+    gp, _ = plans("d5120")
     x = torch.randn(300, 5120, device=DEV, dtype=torch.float32)
     y = gp.apply(x, direction="forward")
     z = gp.apply(y, direction="inverse")
@@ -167,7 +167,7 @@ def _two_sided_plans(u_sched, v_sched, w):
 
 
 def test_two_sided_small_full_compare():
-    w = W.get("c4")
+    w = W.get("two_sided")
     pu, tu, pv, tv = _two_sided_plans((8, 8, 7), (8, 8, 2), w)
     wt = W.draw_encoded(w, 0, 448, 128)
     out = H.apply_two_sided(pu, pv, to_dev(wt))
@@ -180,7 +180,7 @@ def test_two_sided_small_full_compare():
 
 
 def test_two_sided_full_size_sampled_rows():
-    w = W.get("c4")
+    w = W.get("two_sided")
     pu, tu, pv, tv = _two_sided_plans(w.u_schedule, w.schedule, w)
     wt = W.draw_encoded(w, 0, w.n_out, w.n_in)
     out = to_host(H.apply_two_sided(pu, pv, to_dev(wt)))
@@ -203,7 +203,7 @@ def test_two_sided_full_size_sampled_rows():
 
 
 def test_two_sided_in_place():
-    w = W.get("c4")
+    w = W.get("two_sided")
     pu, tu, pv, tv = _two_sided_plans((8, 8, 7), (8, 8, 2), w)
     wt = W.draw_encoded(w, 0, 448, 128)
     t = to_dev(wt)
@@ -216,13 +216,13 @@ def test_two_sided_in_place():
 # --------------------------------------------------------------- edge cases ---
 
 def test_rows_zero_is_a_no_op():
-    gp, _ = plans("c2")
+    gp, _ = plans("d4096")
     x = torch.empty(0, 4096, device=DEV, dtype=torch.bfloat16)
     y = gp.apply(x)
     assert y.shape == (0, 4096)
 
 
-@pytest.mark.parametrize("name", ["c2", "c1"])
+@pytest.mark.parametrize("name", ["d4096", "d64"])
 def test_in_place(name):
     gp, tr = plans(name)
     enc = W.draw_encoded(W.get(name), 0, 129)
@@ -232,7 +232,7 @@ def test_in_place(name):
     check(to_host(x), tr.forward(decode(enc)), decode(enc), f"{name} in place")
 
 
-@pytest.mark.parametrize("name,pad", [("c2", 3), ("c2", 8), ("c1", 1), ("c3", 16)])
+@pytest.mark.parametrize("name,pad", [("d4096", 3), ("d4096", 8), ("d64", 1), ("d5120", 16)])
 def test_leading_dimension_and_guard_bands(name, pad):
     gp, tr = plans(name)
     w = W.get(name)
@@ -259,9 +259,9 @@ def test_leading_dimension_and_guard_bands(name, pad):
 
 
 def test_two_streams_share_a_plan():
-    gp, tr = plans("c2")
-    a = W.draw_encoded(W.get("c2"), 0, 512)
-    b = W.draw_encoded(W.get("c2"), 512, 512)
+    gp, tr = plans("d4096")
+    a = W.draw_encoded(W.get("d4096"), 0, 512)
+    b = W.draw_encoded(W.get("d4096"), 512, 512)
     s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
     xa, xb = to_dev(a), to_dev(b)
     torch.cuda.synchronize()
@@ -275,7 +275,7 @@ def test_two_streams_share_a_plan():
 
 
 def test_partial_overlap_rejected():
-    gp, _ = plans("c2")
+    gp, _ = plans("d4096")
     buf = torch.zeros(8 * 4096 + 4096, device=DEV, dtype=torch.bfloat16)
     x = buf[:8 * 4096].view(8, 4096)
     y = buf[4096:].view(8, 4096)
@@ -285,16 +285,16 @@ def test_partial_overlap_rejected():
 
 
 def test_materialize_is_idempotent_and_blocks_are_reused():
-    gp, tr = plans("c1")
+    gp, tr = plans("d64")
     gp.materialize()
-    enc = full_input("c1", 1024)
+    enc = full_input("d64", 1024)
     out = run(gp, enc, "forward")
     check(out, tr.forward(decode(enc)), decode(enc), "after second materialize")
 
 
 def test_bench_shape_uses_the_specialized_kernel_and_no_wait_gave_up():
-    gp, tr = plans("c2")
-    enc = W.draw_encoded(W.get("c2"), 0, 4096 + 5)
+    gp, tr = plans("d4096")
+    enc = W.draw_encoded(W.get("d4096"), 0, 4096 + 5)
     out = run(gp, enc, "forward")
     assert H.last_kernel() == "harp_fast_d4096_fwd_kernel"
     gp.device_status()

@@ -26,9 +26,9 @@ def tiled(monkeypatch):
 
 
 @pytest.mark.parametrize("name,direction", [
-    ("c1", "forward"), ("c1", "inverse"), ("c1b", "forward"),
-    ("c2", "forward"), ("c2", "inverse"), ("c3", "forward"), ("c3", "inverse"),
-    ("c5", "forward"), ("c5", "inverse")])
+    ("d64", "forward"), ("d64", "inverse"), ("d64_hadamard", "forward"),
+    ("d4096", "forward"), ("d4096", "inverse"), ("d5120", "forward"), ("d5120", "inverse"),
+    ("d8192_int8", "forward"), ("d8192_int8", "inverse")])
 @pytest.mark.parametrize("rows", [1, 5, 37, 300])
 def test_workloads_full_compare(tiled, name, direction, rows):
     gp, tr = plans(name)
@@ -65,7 +65,7 @@ def test_other_radices(tiled, schedule, dtype):
         check(out, tr.apply(xf, direction), xf, f"tiled {schedule} {dtype} {direction}")
 
 
-@pytest.mark.parametrize("name", ["c1", "c3", "c5"])
+@pytest.mark.parametrize("name", ["d64", "d5120", "d8192_int8"])
 def test_same_bits_as_the_simple_kernel(monkeypatch, name):
     """Both kernels sum each output as fma(B[k][l], x_l, acc) over l = 0..b-1 from 0, so
     their fp32 results agree bit for bit."""
@@ -83,7 +83,7 @@ def test_same_bits_as_the_simple_kernel(monkeypatch, name):
         np.testing.assert_array_equal(outs["tiled", direction], outs["simple", direction])
 
 
-@pytest.mark.parametrize("name", ["c3", "c5", "c1"])
+@pytest.mark.parametrize("name", ["d5120", "d8192_int8", "d64"])
 def test_in_place(tiled, name):
     gp, tr = plans(name)
     enc = W.draw_encoded(W.get(name), 0, 23)
@@ -93,7 +93,7 @@ def test_in_place(tiled, name):
     check(to_host(x), tr.inverse(decode(enc)), decode(enc), f"tiled {name} in place")
 
 
-@pytest.mark.parametrize("name,pad", [("c3", 8), ("c5", 64), ("c1", 4)])
+@pytest.mark.parametrize("name,pad", [("d5120", 8), ("d8192_int8", 64), ("d64", 4)])
 def test_padded_rows_and_guard_bands(tiled, name, pad):
     gp, tr = plans(name)
     w = W.get(name)
@@ -127,16 +127,16 @@ def test_shapes_outside_the_tiled_kernel_fall_back(monkeypatch):
     assert e.value.status == HB.HARP_ERR_UNSUPPORTED
 
 
-def test_default_dispatch_takes_the_tiled_kernel_for_c3_and_c5(monkeypatch):
+def test_default_dispatch_takes_the_tiled_kernel_for_d5120_and_c5(monkeypatch):
     monkeypatch.delenv("HARP_KERNEL", raising=False)
-    for name, direction in (("c3", "forward"), ("c5", "inverse"), ("c2", "inverse")):
+    for name, direction in (("d5120", "forward"), ("d8192_int8", "inverse"), ("d4096", "inverse")):
         gp, _ = plans(name)
         run(gp, W.draw_encoded(W.get(name), 0, 64), direction)
         assert H.last_kernel() == "harp_tiled_kernel", name
         gp.device_status()
 
 
-@pytest.mark.parametrize("name", ["c3", "c5"])
+@pytest.mark.parametrize("name", ["d5120", "d8192_int8"])
 @pytest.mark.parametrize("direction", ["forward", "inverse"])
 def test_slab_mode_matches_whole_rows(monkeypatch, name, direction):
     """Slab mode (HARP_TILED_SLAB=1): schedules ending in radix 2 at large d run as CTA pairs

@@ -66,8 +66,8 @@ def test_columns_match_the_transpose_path_bit_for_bit(monkeypatch, n_in_sched):
         np.testing.assert_array_equal(a, b)
 
 
-def test_full_size_c4_matches_the_transpose_path_on_sampled_rows(monkeypatch):
-    w4 = W.get("c4")
+def test_full_size_two_sided_matches_the_transpose_path_on_sampled_rows(monkeypatch):
+    w4 = W.get("two_sided")
     pu, _ = _pair(w4.u_schedule, 71)
     pv, _ = _pair(w4.schedule, 72)
     wt = to_dev(W.draw_encoded(w4, 0, w4.n_out, w4.n_in))

@@ -8,21 +8,23 @@ be regenerated on its own without drawing the rest.
 Workloads (HARP, "Technical Summary: HARP", sections 2.1-2.4; the shapes and
 value distributions are the ones the five workload definitions name):
 
-* ``c1``   d=64, schedule (8,8), 1024 rows fp32, x iid N(0,1), theta ~ N(0, 0.1)
-* ``c1b``  d=64, schedule (2,2,2,2,2,2), theta = 0 (the fixed randomized Hadamard)
-* ``c2``   d=4096, (8,8,8,8), 65,536 rows bf16, Student-t (nu=3) entries with 8
+* ``d64``   d=64, schedule (8,8), 1024 rows fp32, x iid N(0,1), theta ~ N(0, 0.1)
+* ``d64_hadamard``  d=64, schedule (2,2,2,2,2,2), theta = 0 (the fixed randomized Hadamard)
+* ``d4096``   d=4096, (8,8,8,8), 65,536 rows bf16, Student-t (nu=3) entries with 8
            seeded outlier channels x50, theta ~ N(0, 0.05), forward
-* ``c3``   d=5120, (8,8,8,5,2), 32,768 rows bf16, N(0,1) with 1% of entries x20,
-           theta ~ N(0, 0.05), forward and inverse (``c3_64k``: 65,536 rows)
-* ``c4``   two-sided U^T W V: W 28672x8192 bf16 iid N(0, 0.02^2) with 16 outlier
+* ``d5120``   d=5120, (8,8,8,5,2), 32,768 rows bf16, N(0,1) with 1% of entries x20,
+           theta ~ N(0, 0.05), forward and inverse (``d5120_64k``: 65,536 rows)
+* ``two_sided``   two-sided U^T W V: W 28672x8192 bf16 iid N(0, 0.02^2) with 16 outlier
            columns x30; U (8,8,8,8,7), V (8,8,8,8,2), theta ~ N(0, 0.05)
-* ``c5``   d=8192, (8,8,8,8,2), int8 theta + per-stage fp32 scale, bf16 rows in
+* ``d8192_int8``   d=8192, (8,8,8,8,2), int8 theta + per-stage fp32 scale, bf16 rows in
            {1, 16, 256, 65536}, iid N(0,1), forward and inverse
 
 "N(0, v)" is read as variance v (the same workload list writes the weight
 distribution as N(0, 0.02^2)), so theta's standard deviation is sqrt(v).
 
-Seeds: data = 1000 + k, theta = 2000 + k, sign seed = 3000 + k for workload k.
+Seeds: data = 1000 + k, theta = 2000 + k, sign seed = 3000 + k, where k is the
+workload's seed index (1 for d64 and d64_hadamard, 2 for d4096, 3 for d5120 and
+d5120_64k, 4 for two_sided, 5 for d8192_int8).
 """
 from __future__ import annotations
 
@@ -37,7 +39,7 @@ import numpy as np
 ROW_BLOCK = 256
 
 __all__ = [
-    "ROW_BLOCK", "Workload", "CONFIGS", "get", "draw_rows", "draw_theta",
+    "ROW_BLOCK", "Workload", "WORKLOADS", "get", "draw_rows", "draw_theta",
     "encode_bf16", "decode_bf16", "quantize_theta_int8", "sample_rows",
     "draw_weight", "draw_encoded", "C5_ROWS",
 ]
@@ -80,21 +82,21 @@ class Workload:
 _S01 = math.sqrt(0.1)
 _S005 = math.sqrt(0.05)
 
-CONFIGS = {
-    "c1": Workload("c1", 1, 64, (8, 8), 1024, "f32", "normal", _S01,
+WORKLOADS = {
+    "d64": Workload("d64", 1, 64, (8, 8), 1024, "f32", "normal", _S01,
                    dirs=("forward", "inverse")),
-    "c1b": Workload("c1b", 1, 64, (2, 2, 2, 2, 2, 2), 1024, "f32", "normal", 0.0),
-    "c2": Workload("c2", 2, 4096, (8, 8, 8, 8), 65536, "bf16", "student_t_outlier_channels",
+    "d64_hadamard": Workload("d64_hadamard", 1, 64, (2, 2, 2, 2, 2, 2), 1024, "f32", "normal", 0.0),
+    "d4096": Workload("d4096", 2, 4096, (8, 8, 8, 8), 65536, "bf16", "student_t_outlier_channels",
                    _S005),
-    "c3": Workload("c3", 3, 5120, (8, 8, 8, 5, 2), 32768, "bf16", "normal_sparse_x20",
+    "d5120": Workload("d5120", 3, 5120, (8, 8, 8, 5, 2), 32768, "bf16", "normal_sparse_x20",
                    _S005, dirs=("forward", "inverse")),
-    "c3_64k": Workload("c3_64k", 3, 5120, (8, 8, 8, 5, 2), 65536, "bf16",
+    "d5120_64k": Workload("d5120_64k", 3, 5120, (8, 8, 8, 5, 2), 65536, "bf16",
                        "normal_sparse_x20", _S005, dirs=("forward", "inverse")),
     # two-sided: rows of W get the V side (d = n_in), columns the U side (d = n_out)
-    "c4": Workload("c4", 4, 8192, (8, 8, 8, 8, 2), 28672, "bf16", "weight_outlier_columns",
+    "two_sided": Workload("two_sided", 4, 8192, (8, 8, 8, 8, 2), 28672, "bf16", "weight_outlier_columns",
                    _S005, dirs=("two_sided",), u_schedule=(8, 8, 8, 8, 7),
                    n_out=28672, n_in=8192),
-    "c5": Workload("c5", 5, 8192, (8, 8, 8, 8, 2), 65536, "bf16", "normal", _S005,
+    "d8192_int8": Workload("d8192_int8", 5, 8192, (8, 8, 8, 8, 2), 65536, "bf16", "normal", _S005,
                    theta_kind="i8", dirs=("forward", "inverse")),
 }
 
@@ -102,7 +104,7 @@ C5_ROWS = (1, 16, 256, 65536)
 
 
 def get(name: str, rows: Optional[int] = None) -> Workload:
-    w = CONFIGS[name]
+    w = WORKLOADS[name]
     if rows is not None:
         w = dataclasses.replace(w, rows=int(rows))
     return w
