@@ -49,7 +49,7 @@ def log(*a):
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="d4096", choices=["d4096", "d5120_64k", "d8192_int8"])
@@ -365,6 +365,21 @@ def side_measurements(args, H, W, torch, device, peak):
                     "traffic": recorded_traffic(kn, name) if direction == "forward" else None})
         del y2
     cache.clear()
+    # decode-shaped batches of the d = 8192 int8 workload: latency of one call
+    wd = W.get("d8192_int8")
+    pd_ = make_plan("d8192_int8", H, W)
+    for rows_d in (1, 16, 256):
+        xd = to_device_bf16(W.draw_encoded(wd, 0, rows_d), torch, device)
+        yd = torch.empty_like(xd)
+        for direction in ("forward", "inverse"):
+            st = 200
+            el, km, _, kn = time_apply(pd_, xd, yd, st, 20, torch, direction=direction)
+            out.append({"workload": f"d=8192 schedule (8,8,8,8,2), int8 theta, {rows_d} bf16 rows (decode-shaped), "
+                                    f"{direction}", "rows_per_s": rows_d * st / (el / 1e3),
+                        "us_per_call": 1e3 * el / st, "kernel": kn, "kernel_ms": km,
+                        "hbm_frac": 4 * rows_d * wd.d / (km / 1e3) / 1e9 / peak})
+        del xd, yd
+    del pd_
     # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)
     w4 = W.get("two_sided")
     th_v = W.draw_theta(H.theta_count(w4.schedule), w4.theta_sigma, w4.theta_seed)

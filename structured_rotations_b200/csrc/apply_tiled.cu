@@ -120,6 +120,19 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
             }
         }
     }
+    // Small batches (decode-shaped): 4-row sub-tiles would pad rows with zeros and leave
+    // most SMs idle, so one-row sub-tiles spread the rows over as many SMs as possible.
+    if (cl == 1 && sh.V == 4 && rows < 4 * (int64_t)sm_count() && has_row_major_kernel(kMasks[which])) {
+        const char* env = std::getenv("HARP_TILED_SMALL");
+        if (!(env && !std::strcmp(env, "0"))) {
+            const int64_t r1 = std::min<int64_t>((rows + sm_count() - 1) / sm_count(), budget / (4 * d));
+            if (r1 >= 1) {
+                sh.V = 1;
+                sh.R = r1;
+                sh.staged = std::max<int64_t>(0, std::min<int64_t>(r1, (budget - r1 * d * 4) / (d * es_in)));
+            }
+        }
+    }
     const int V = sh.V;
     const int64_t R = sh.R, staged = sh.staged, dl = d / cl;
     if (R < 1 || (V == 1 && !has_row_major_kernel(kMasks[which]))) return HARP_ERR_UNSUPPORTED;
