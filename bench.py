@@ -314,6 +314,35 @@ def time_apply(plan, x, y, steps, warmup, torch, dist=None, direction="forward")
     return elapsed, kern, steps, H.last_kernel()
 
 
+def time_calls(plan, x, y, calls, warmup, torch, direction):
+    """Per-call cost of small launches, three ways (microseconds): on the device, with the
+    stream held back by a sleep kernel so that all `calls` launches are queued before the
+    first runs (launch gaps included, host time excluded); on the host, the time the public
+    call takes to return while the device is busy; and the wall time per call of `calls`
+    back-to-back calls followed by one synchronize."""
+    import structured_rotations_b200 as H
+    for _ in range(warmup):
+        plan.apply(x, y, direction=direction)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e8))          # about 0.1 s at the B200's clock: longer than the submissions
+    e0.record(stream)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        plan.apply(x, y, direction=direction)
+    host_us = (time.perf_counter() - t0) * 1e6 / calls
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dev_us = e0.elapsed_time(e1) * 1e3 / calls
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        plan.apply(x, y, direction=direction)
+    torch.cuda.synchronize()
+    wall_us = (time.perf_counter() - t0) * 1e6 / calls
+    return dev_us, host_us, wall_us, H.last_kernel()
+
+
 def end_to_end(args, plan, enc, x, y, torch, dist, device, world, rows):
     """The same metric through the public host-buffer call (harp_apply_host): every step
     copies this rank's rows from pinned host memory to the GPU, rotates them and copies
@@ -365,19 +394,18 @@ def side_measurements(args, H, W, torch, device, peak):
                     "traffic": recorded_traffic(kn, name) if direction == "forward" else None})
         del y2
     cache.clear()
-    # decode-shaped batches of the d = 8192 int8 workload: latency of one call
+    # decode-shaped batches of the d = 8192 int8 workload: cost of one call
     wd = W.get("d8192_int8")
     pd_ = make_plan("d8192_int8", H, W)
     for rows_d in (1, 16, 256):
         xd = to_device_bf16(W.draw_encoded(wd, 0, rows_d), torch, device)
         yd = torch.empty_like(xd)
         for direction in ("forward", "inverse"):
-            st = 200
-            el, km, _, kn = time_apply(pd_, xd, yd, st, 20, torch, direction=direction)
+            dev_us, host_us, wall_us, kn = time_calls(pd_, xd, yd, 200, 20, torch, direction)
             out.append({"workload": f"d=8192 schedule (8,8,8,8,2), int8 theta, {rows_d} bf16 rows (decode-shaped), "
-                                    f"{direction}", "rows_per_s": rows_d * st / (el / 1e3),
-                        "us_per_call": 1e3 * el / st, "kernel": kn, "kernel_ms": km,
-                        "hbm_frac": 4 * rows_d * wd.d / (km / 1e3) / 1e9 / peak})
+                                    f"{direction}", "rows_per_s": rows_d / (wall_us / 1e6),
+                        "us_per_call": wall_us, "device_us_per_call": dev_us, "host_us_per_call": host_us,
+                        "kernel": kn, "hbm_frac": 4 * rows_d * wd.d / (dev_us / 1e6) / 1e9 / peak})
         del xd, yd
     del pd_
     # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)

@@ -3,6 +3,9 @@
 // (HARP abstract: a two-sided orthogonal processor; W_out = T_U^T W T_V).
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include <cuda_runtime.h>
 
@@ -25,8 +28,8 @@ harp_status check_device(const harp_plan_s* p) {
 }
 
 // HARP_KERNEL selects the row kernel: unset = the fastest one that covers the shape
-// (specialized, then tiled, then simple); "simple", "tiled" or "fast" (specialized)
-// force one and fail with HARP_ERR_UNSUPPORTED if it does not cover the shape.
+// (specialized, then tiled, then simple); "simple", "tiled" or "fast" (specialized) force
+// one and fail with HARP_ERR_UNSUPPORTED if it does not cover the shape.
 enum { kAuto = 0, kSimple = 1, kFast = 2, kTiled = 3 };
 
 int kernel_choice() {
@@ -39,6 +42,19 @@ int kernel_choice() {
 }
 
 }  // namespace
+
+int harp_set_smem_limit(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, int> done;   // (device, kernel) -> limit set
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find({dev, kernel});
+    if (it != done.end() && it->second >= bytes) return (int)cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[{dev, kernel}] = bytes;
+    return (int)e;
+}
 
 // The row kernels in order of preference.
 harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x, int64_t ld_y,

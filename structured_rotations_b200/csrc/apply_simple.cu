@@ -98,7 +98,7 @@ harp_status launch_typed(const harp_plan_s* p, const void* x, void* y, int64_t r
     const size_t smem = row_bytes * rpc;
     auto kern = apply_simple_kernel<TIn, TOut>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = (cudaError_t)harp_set_smem_limit((const void*)kern, (int)smem);
         if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     }
     const int64_t grid = (rows + rpc - 1) / rpc;

@@ -555,7 +555,7 @@ cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid,
             return cudaErrorInvalidValue;
         } else {
             auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT, CL>;
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaError_t e = (cudaError_t)harp_set_smem_limit((const void*)kern, (int)smem);
             if (e != cudaSuccess) return e;
             if constexpr (CL == 1) {
                 kern<<<(unsigned)grid, NT, smem, stream>>>(tp);

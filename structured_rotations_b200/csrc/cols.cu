@@ -305,7 +305,7 @@ harp_status launch_cols(const harp_plan_s* pl, float* x, int64_t ld_x, int64_t n
         cp.out_bf16 = last && out_dtype == HARP_BF16;
         const int row_tiles = a ? P / PB : Q / SB;
         const size_t smem = (size_t)(a ? PB * Q * row_a : SB * P * row_b);
-        cudaError_t e = cudaFuncSetAttribute(harp_cols_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = (cudaError_t)harp_set_smem_limit((const void*)harp_cols_kernel, (int)smem);
         if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
         const int64_t grid = (int64_t)row_tiles * col_tiles;
         if (grid > 0x7fffffff) return HARP_ERR_UNSUPPORTED;

@@ -62,6 +62,10 @@ struct harp_plan_s {
 harp_status harp_fail(harp_status s, const std::string& msg);
 void harp_clear_error();
 void harp_set_last_kernel(const char* name);
+// Raises a kernel's dynamic shared-memory limit (cudaFuncAttributeMaxDynamicSharedMemorySize)
+// to at least `bytes` on the current device; the runtime call is made only the first time a
+// kernel needs more than before, since it costs microseconds on every launch otherwise.
+int harp_set_smem_limit(const void* kernel, int bytes);
 
 // device helpers (materialize.cu)
 harp_status harp_device_free(harp_plan_s* p);

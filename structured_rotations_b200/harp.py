@@ -119,6 +119,9 @@ def splitmix64(seed: int, n: int) -> np.ndarray:
 def _stream_handle(stream) -> Optional[int]:
     if stream is None:
         import torch
+        C = torch._C
+        if hasattr(C, "_cuda_getCurrentRawStream"):   # the handle without a Stream object
+            return C._cuda_getCurrentRawStream(C._cuda_getDevice())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
         return stream
@@ -128,11 +131,17 @@ def _stream_handle(stream) -> Optional[int]:
 _DTYPE = {"float32": HARP_F32, "bfloat16": HARP_BF16}
 
 
+_DTYPE_OF = {}   # torch dtype -> code, filled on first use
+
+
 def _dtype_code(t) -> int:
-    name = str(t.dtype).replace("torch.", "")
-    if name not in _DTYPE:
-        raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
-    return _DTYPE[name]
+    code = _DTYPE_OF.get(t.dtype)
+    if code is None:
+        name = str(t.dtype).replace("torch.", "")
+        if name not in _DTYPE:
+            raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+        code = _DTYPE_OF[t.dtype] = _DTYPE[name]
+    return code
 
 
 def _ld(t) -> int:
