@@ -331,3 +331,107 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 def round_f32(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Calibration backward: the gradient of a loss with respect to theta
+# ---------------------------------------------------------------------------
+#
+# HARP is fitted per layer from calibration data by minimizing a surrogate loss
+# (§2.3 Optimization Objective), so a fit needs dL/dtheta through the transform.
+# For rows x_r with upstream gradients g_r = dL/dy_r of y_r = T x_r, the loss is
+# locally L = sum_r g_r . (T x_r) and its gradient is built here from the chain
+# rule, step by step:
+#
+#   z_0 = S x, z_{t+1} = M_t z_t        (stage inputs, forward)
+#   h_m = g,   h_t = M_t^T h_{t+1}      (gradients at the stage inputs, backward)
+#   dL/dB_{t,c}[k][l] = sum_r h_{t+1,r}[lo + s_t (k + b_t hi)] z_{t,r}[lo + s_t (l + b_t hi)]
+#   dL/dQ = dL/dB G^T                   (B = Q G)
+#   Givens: dL/dtheta = sum dL/dQ * dQ/dtheta, dQ/dtheta = [[-sin, -cos], [cos, -sin]]
+#   Cayley: Q = M (I + A) with M = (I - A)^{-1}, so dQ = M dA (Q + I) and
+#           dL/dA = M^T dL/dQ (Q + I)^T; theta_k sits at A[i][j] = theta_k and
+#           A[j][i] = -theta_k, so dL/dtheta_k = dL/dA[i][j] - dL/dA[j][i].
+#
+# dL/dx itself is T^T g, the inverse transform.  For int8 storage the gradient is
+# taken with respect to the dequantized values q * scale_t.
+
+def block_grads(plan: OraclePlan, x: np.ndarray, g: np.ndarray) -> List[np.ndarray]:
+    """dL/dB_{t,c} for L = sum_r g_r . (T x_r): per stage an array [d/b_t, b_t, b_t]."""
+    tr = Transform(plan)
+    z = np.asarray(x, dtype=np.float64) * tr.signs[None, :]
+    inputs = []
+    for mt in tr.mats:
+        inputs.append(z)
+        z = (mt @ z.T).T
+    h = np.asarray(g, dtype=np.float64)
+    out = [None] * plan.m
+    for t in reversed(range(plan.m)):
+        b, s = plan.schedule[t], strides(plan.schedule)[t]
+        zt = inputs[t]
+        gb = np.zeros((plan.d // b, b, b))
+        for c in range(plan.d // b):
+            lo, hi = c % s, c // s
+            idx = [lo + s * (k + b * hi) for k in range(b)]
+            gb[c] = h[:, idx].T @ zt[:, idx]          # sum over rows of h[k] z[l]
+        out[t] = gb
+        h = (tr.mats[t].T @ h.T).T
+    return out
+
+
+def theta_grad_from_blocks(plan: OraclePlan, dblocks: List[np.ndarray]) -> np.ndarray:
+    """dL/dtheta from dL/dB_{t,c} through B = Q(theta) G (Givens or Cayley)."""
+    out = np.empty(theta_count(plan.schedule))
+    off = 0
+    for t, b in enumerate(plan.schedule):
+        g = base_mixer(b, plan.qr_seed)
+        p = params_per_block(b)
+        for c in range(plan.d // b):
+            par = plan.theta[off + c * p: off + (c + 1) * p]
+            dq = dblocks[t][c] @ g.T
+            if b == 2:
+                cs, sn = math.cos(par[0]), math.sin(par[0])
+                out[off + c] = np.sum(dq * np.array([[-sn, -cs], [cs, -sn]]))
+            else:
+                a = skew_from_params(par, b)
+                eye = np.eye(b)
+                minv = np.linalg.inv(eye - a)
+                q = minv @ (eye + a)
+                da = minv.T @ dq @ (q + eye).T
+                k = 0
+                for i in range(b):
+                    for j in range(i + 1, b):
+                        out[off + c * p + k] = da[i, j] - da[j, i]
+                        k += 1
+        off += (plan.d // b) * p
+    return out
+
+
+def theta_grad(plan: OraclePlan, x: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """dL/dtheta for L = sum_r g_r . (T(theta) x_r), in the theta layout of the plan."""
+    return theta_grad_from_blocks(plan, block_grads(plan, x, g))
+
+
+def theta_grad_scale(plan: OraclePlan, x: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """Per parameter, sum_r |h_{t+1,r}[group]| |z_{t,r}[group]| over the rows for the
+    parameter's block: every entry of dL/dB_{t,c} is at most this in magnitude, and
+    |dL/dtheta| at most 4 times it (|M| <= 1, |Q + I| <= 2, G orthogonal, two entries
+    per parameter).  Used to scale comparison tolerances."""
+    tr = Transform(plan)
+    z = np.asarray(x, dtype=np.float64) * tr.signs[None, :]
+    inputs = []
+    for mt in tr.mats:
+        inputs.append(z)
+        z = (mt @ z.T).T
+    h = np.asarray(g, dtype=np.float64)
+    per_stage = [None] * plan.m
+    for t in reversed(range(plan.m)):
+        b, s = plan.schedule[t], strides(plan.schedule)[t]
+        zt = inputs[t]
+        sc = np.zeros(plan.d // b)
+        for c in range(plan.d // b):
+            lo, hi = c % s, c // s
+            idx = [lo + s * (k + b * hi) for k in range(b)]
+            sc[c] = np.sum(np.linalg.norm(h[:, idx], axis=1) * np.linalg.norm(zt[:, idx], axis=1))
+        per_stage[t] = sc
+        h = (tr.mats[t].T @ h.T).T
+    return np.concatenate([np.repeat(per_stage[t], params_per_block(b)) for t, b in enumerate(plan.schedule)])
