@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--workload", default="d4096", choices=["d4096", "d5120_64k", "d8192_int8"])
     ap.add_argument("--no-extra", action="store_true", help="skip the d=5120 / d=8192 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grad-rows", type=int, default=0,
+                    help="time only the calibration backward (harp_grad_theta) on this many d=4096 rows and "
+                         "print its line (for profiling that kernel alone)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--rows", type=int, default=0, help="rows per GPU (default: the workload's; "
@@ -436,6 +439,54 @@ def side_measurements(args, H, W, torch, device, peak):
     return out
 
 
+def grad_roofline(res, clocks, device, torch):
+    """The FMA roofline of a grad_measurement line at the sampled median SM clock (the
+    maximum clock if none was sampled)."""
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    alu_peak = sms * 128 * mhz * 1e6
+    res["roofline"] = {"bound": "alu", "achieved": res["fma_per_s"] / 1e12, "peak": alu_peak / 1e12,
+                       "unit": "TFMA/s", "frac": res["fma_per_s"] / alu_peak,
+                       "peak_source": f"{sms} SMs x 128 FP32 lanes x {mhz} MHz (median sampled SM clock)"}
+    return res
+
+
+def grad_measurement(H, W, torch, device, peak, rows=None, steps=10):
+    """The calibration backward dL/dtheta (harp_grad_theta) on the d = 4096 workload: rows
+    x and upstream gradients g (bf16, N(0, 1)), device-timed over `steps` calls (each
+    call: accumulator reset, the block-gradient kernel, the theta kernel).  Its roof is
+    the FP32 FMA rate: 4 d sum(b) FMA per row (the forward chain once, the backward
+    chain's two transposed products and the outer product) against 148 SMs x 128 FMA
+    lanes at the sampled SM clock; it reads 4 d bytes per row from HBM."""
+    w = W.get("d4096")
+    rows = rows or w.rows
+    plan = make_plan("d4096", H, W)
+    x = to_device_bf16(W.draw_encoded(w, 0, rows), torch, device)
+    g = to_device_bf16(W.draw_upstream(w, 0, rows), torch, device)
+    out = torch.empty(H.theta_count(w.schedule), dtype=torch.float32, device=device)
+    ws = torch.empty(int(H.lib().harp_grad_workspace_bytes(plan.handle)), dtype=torch.uint8, device=device)
+    for _ in range(3):
+        plan.grad_theta(x, g, out, ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        plan.grad_theta(x, g, out, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    fma = 4 * w.d * sum(w.schedule) * rows
+    byt = 4 * rows * w.d
+    return {"workload": f"calibration backward dL/dtheta, d=4096 schedule (8,8,8,8), {rows} bf16 rows x and "
+                        f"upstream gradients g (N(0,1)), theta~N(0,0.05)",
+            "ms": ms, "rows_per_s": rows / (ms / 1e3), "hbm_gbs": byt / (ms / 1e3) / 1e9,
+            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "fma_per_row": 4 * w.d * sum(w.schedule),
+            "fma_per_s": fma / (ms / 1e3),
+            "kernel": "harp_grad_blocks_kernel + harp_grad_theta_kernel", "steps": steps,
+            "traffic": (recorded_traffic("harp_grad_blocks_kernel", "d4096") if rows == w.rows else None)}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -456,6 +507,15 @@ def run_ours(args):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=device)
         dist = tdist
+
+    if args.grad_rows:
+        peak, _ = peaks()
+        sampler = ClockSampler(local)
+        sampler.start()
+        res = grad_measurement(H, W, torch, device, peak, args.grad_rows, args.steps)
+        clocks = sampler.stop()
+        print(json.dumps(grad_roofline(res, clocks, device, torch)))
+        return 0
 
     w = W.get(args.workload, args.rows or None)
     rows, d = w.rows, w.d
@@ -486,6 +546,7 @@ def run_ours(args):
     also = []
     if not args.no_extra and rank == 0 and world == 1:
         also = side_measurements(args, H, W, torch, device, peak)
+        also.append(grad_roofline(grad_measurement(H, W, torch, device, peak), clocks, device, torch))
 
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and world == 1:

@@ -233,6 +233,37 @@ HARP_API harp_status harp_apply_two_sided_noalloc(harp_plan_t planU, harp_plan_t
 /* harp_noalloc_scratch_bytes — size of that static array (HARP_NOALLOC_SCRATCH_BYTES). */
 HARP_API size_t harp_noalloc_scratch_bytes(void);
 
+/*
+ * harp_grad_workspace_bytes — device workspace that harp_grad_theta needs for this plan:
+ * one float accumulator per block entry (4 d sum_t b_t bytes, each stage padded to 16
+ * bytes).  0 for a NULL plan.
+ */
+HARP_API size_t harp_grad_workspace_bytes(harp_plan_t plan);
+
+/*
+ * harp_grad_theta — calibration backward (§2.3 Optimization Objective: theta is fitted
+ * per layer from calibration data): dtheta = dL/dtheta for L = sum_r g_r . (T x_r), i.e.
+ * the gradient of a loss through the forward transform given the upstream gradients
+ * g_r = dL/dy_r.  (dL/dx_r = T^T g_r is harp_apply with HARP_INVERSE.)
+ *   x, g        device pointers, rows of d elements of type dtype (both the same type),
+ *               leading dimensions ld_x, ld_g >= d.
+ *   rows        number of rows; 0 writes dtheta = 0.
+ *   dtheta      device float array of the plan's theta count, overwritten, in the theta
+ *               layout of harp_plan_create (stages in order, blocks in c order, the
+ *               block's parameters contiguous).  For int8 plans it is the gradient with
+ *               respect to the dequantized values q * scale_t.
+ *   workspace   device memory of at least harp_grad_workspace_bytes(plan) bytes,
+ *               16-byte aligned; overwritten.
+ * Arithmetic: fp32 in the stage chain and the per-tile sums, fp32 atomic additions across
+ * tiles (the order of those additions varies between runs, so the last bits of dtheta
+ * may too), double in the map from block gradients to theta.
+ * Returns HARP_ERR_UNSUPPORTED for radices above 8 and for rows too long for two fp32 rows
+ * in shared memory (d above 29,056); asynchronous on `stream` like harp_apply.
+ */
+HARP_API harp_status harp_grad_theta(harp_plan_t plan, const void* x, const void* g, int64_t rows,
+                                     int64_t ld_x, int64_t ld_g, harp_dtype dtype, float* dtheta,
+                                     void* workspace, size_t ws_bytes, void* stream);
+
 /* harp_plan_device_status — synchronizes the plan's device and reports whether any
  * bounded device-side wait of a kernel launched with this plan gave up since the
  * last call: HARP_ERR_TIMEOUT if one did (the flag is then cleared), HARP_OK if

@@ -73,6 +73,9 @@ def lib():
                                                   _vp]),
         "harp_noalloc_scratch_bytes": (ctypes.c_size_t, []),
         "harp_plan_device_status": (_c_i32, [_vp]),
+        "harp_grad_workspace_bytes": (ctypes.c_size_t, [_vp]),
+        "harp_grad_theta": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _vp, ctypes.c_size_t,
+                                     _vp]),
         "harp_plan_destroy": (_c_i32, [_vp]),
         "harp_status_string": (ctypes.c_char_p, [_c_i32]),
         "harp_last_error": (ctypes.c_char_p, []),
@@ -203,6 +206,28 @@ class Plan:
         _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
                                 _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
         return y
+
+    def grad_theta(self, x, g, dtheta=None, workspace=None, stream=None):
+        """dL/dtheta for L = sum_r g_r . (T x_r) (harp_grad_theta): the calibration backward
+        through the forward transform, for rows x and upstream gradients g = dL/dy of one
+        dtype on the GPU.  Returns a float32 tensor of theta_count entries (dtheta, if
+        given, is filled).  dL/dx is self.apply(g, direction="inverse")."""
+        import torch
+        if x.dtype != g.dtype or x.shape != g.shape or x.shape[-1] != self.d:
+            raise ValueError(f"x and g must be rows of d={self.d} of one dtype")
+        n = theta_count(self.schedule)
+        if dtheta is None:
+            dtheta = torch.empty(n, dtype=torch.float32, device=x.device)
+        if dtheta.dtype != torch.float32 or dtheta.numel() != n or not dtheta.is_contiguous():
+            raise ValueError(f"dtheta must be a contiguous float32 tensor of {n} entries")
+        need = int(lib().harp_grad_workspace_bytes(self._h))
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        _check(lib().harp_grad_theta(self._h, x.data_ptr(), g.data_ptr(), x.shape[0], _ld(x), _ld(g),
+                                     _dtype_code(x), dtheta.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), _stream_handle(stream)),
+               "harp_grad_theta")
+        return dtheta
 
     def apply_host(self, x, y=None, direction: str = "forward"):
         """Rows of a host (CPU) tensor through the GPU and back (harp_apply_host): copies,

@@ -41,7 +41,7 @@ ROW_BLOCK = 256
 __all__ = [
     "ROW_BLOCK", "Workload", "WORKLOADS", "get", "draw_rows", "draw_theta",
     "encode_bf16", "decode_bf16", "quantize_theta_int8", "sample_rows",
-    "draw_weight", "draw_encoded", "C5_ROWS",
+    "draw_weight", "draw_encoded", "draw_upstream", "C5_ROWS",
 ]
 
 
@@ -254,6 +254,27 @@ def _encode_threads(x: np.ndarray) -> np.ndarray:
 
     with cf.ThreadPoolExecutor(max_workers=_threads()) as ex:
         list(ex.map(one, parts))
+    return out
+
+
+def draw_upstream(w: Workload, row_start: int = 0, row_count: Optional[int] = None) -> np.ndarray:
+    """Upstream gradients dL/dy for the calibration backward, rows [row_start,
+    row_start+row_count) of i.i.d. N(0, 1) draws in the workload's storage form (float32
+    or bf16 bit patterns), from a stream of their own keyed by [data seed, 0x6AD, block]."""
+    if row_count is None:
+        row_count = w.rows - row_start
+    out = np.empty((row_count, w.d), dtype=np.uint16 if w.dtype == "bf16" else np.float32)
+    first, last = row_start // ROW_BLOCK, (row_start + row_count - 1) // ROW_BLOCK if row_count else -1
+
+    def one(blk):
+        rng = np.random.default_rng([w.data_seed, 0x6AD, blk])
+        x = rng.standard_normal((ROW_BLOCK, w.d))
+        a, b = max(row_start, blk * ROW_BLOCK), min(row_start + row_count, (blk + 1) * ROW_BLOCK)
+        part = x[a - blk * ROW_BLOCK:b - blk * ROW_BLOCK]
+        out[a - row_start:b - row_start] = encode_bf16(part) if w.dtype == "bf16" else part.astype(np.float32)
+
+    with cf.ThreadPoolExecutor(max_workers=_threads()) as ex:
+        list(ex.map(one, range(first, last + 1)))
     return out
 
 
