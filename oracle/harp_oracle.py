@@ -435,3 +435,27 @@ def theta_grad_scale(plan: OraclePlan, x: np.ndarray, g: np.ndarray) -> np.ndarr
         per_stage[t] = sc
         h = (tr.mats[t].T @ h.T).T
     return np.concatenate([np.repeat(per_stage[t], params_per_block(b)) for t, b in enumerate(plan.schedule)])
+
+
+# ---------------------------------------------------------------------------
+# Blockwise quantizer on the rotated rows (fused epilogue)
+# ---------------------------------------------------------------------------
+#
+# HARP is a drop-in preprocessing step in front of a blockwise quantizer (§2.4
+# Deployment Efficiency; §2.3: the fit targets the deployed blockwise quantizer), so
+# the rotated rows are quantized right away.  The quantizer here is the plain
+# symmetric round-to-nearest one: per aligned block of qblock coordinates of a row,
+# s = max |y| / 127 and q = clamp(round_half_even(y / s), -127, 127); s = 0 and
+# q = 0 for an all-zero block.
+
+def quantize_blocks(y: np.ndarray, qblock: int):
+    """(int8 codes [rows, d], float64 scales [rows, d / qblock]) of rows y."""
+    y = np.asarray(y, dtype=np.float64)
+    rows, d = y.shape
+    if d % qblock:
+        raise ValueError("qblock must divide d")
+    yb = y.reshape(rows, d // qblock, qblock)
+    s = np.max(np.abs(yb), axis=2) / 127.0
+    safe = np.where(s > 0, s, 1.0)
+    q = np.where(s[..., None] > 0, np.rint(yb / safe[..., None]), 0.0)
+    return np.clip(q, -127, 127).astype(np.int8).reshape(rows, d), s
