@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--workload", default="d4096", choices=["d4096", "d5120_64k", "d8192_int8"])
     ap.add_argument("--no-extra", action="store_true", help="skip the d=5120 / d=8192 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant-rows", type=int, default=0,
+                    help="time only the fused rotate-then-quantize pass (harp_apply_quant) on this many d=4096 "
+                         "rows and print its line (for profiling that kernel alone)")
     ap.add_argument("--grad-rows", type=int, default=0,
                     help="time only the calibration backward (harp_grad_theta) on this many d=4096 rows and "
                          "print its line (for profiling that kernel alone)")
@@ -436,7 +439,36 @@ def side_measurements(args, H, W, torch, device, peak):
     out.append({"workload": WORKLOAD_TEXT["two_sided"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
                 "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
     del wt, wo, ws
+    out.append(quant_measurement(args, H, W, torch, device, peak))
     return out
+
+
+def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):
+    """The fused rotate-then-quantize pass (harp_apply_quant) on the d = 4096 workload:
+    bf16 rows in, int8 codes and one fp32 scale per 128 coordinates out; algorithmic HBM
+    bytes 2 d + d + 4 d / qblock per row."""
+    w = W.get("d4096", rows)
+    plan = make_plan("d4096", H, W)
+    x = to_device_bf16(W.draw_encoded(w, 0, w.rows), torch, device)
+    q = torch.empty(w.rows, w.d, dtype=torch.int8, device=device)
+    sc = torch.empty(w.rows, w.d // qblock, dtype=torch.float32, device=device)
+    for _ in range(3):
+        plan.apply_quant(x, qblock, q=q, scales=sc)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    st = max(3, args.steps // 4)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(st)]
+    for a, b in ev:
+        a.record(stream)
+        plan.apply_quant(x, qblock, q=q, scales=sc)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    byt = w.rows * (2 * w.d + w.d + 4 * (w.d // qblock))
+    return {"workload": f"rotate + int8 quantize (qblock {qblock}): d=4096 schedule (8,8,8,8), {w.rows} bf16 rows "
+                        f"-> int8 codes + fp32 scales, forward",
+            "kernel_ms": ms, "rows_per_s": w.rows / (ms / 1e3), "hbm_gbs": byt / (ms / 1e3) / 1e9,
+            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": H.last_kernel() + " (int8 epilogue)"}
 
 
 def grad_roofline(res, clocks, device, torch):
@@ -508,6 +540,10 @@ def run_ours(args):
                                  device_id=device)
         dist = tdist
 
+    if args.quant_rows:
+        peak, _ = peaks()
+        print(json.dumps(quant_measurement(args, H, W, torch, device, peak, rows=args.quant_rows)))
+        return 0
     if args.grad_rows:
         peak, _ = peaks()
         sampler = ClockSampler(local)

@@ -164,6 +164,30 @@ HARP_API harp_status harp_apply_host(harp_plan_t plan, const void* x, void* y, i
                                      int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir);
 
 /*
+ * harp_apply_quant — the row transform with a fused blockwise quantizer on its output
+ * (the rotated rows feed a blockwise quantizer: §2.4, a drop-in preprocessing step in
+ * front of the quantizer backend).  For every row r and every aligned block of `qblock`
+ * coordinates of y_r = T x_r (FORWARD) or T^T x_r (INVERSE), computed in fp32 as in
+ * harp_apply:
+ *   s = a / 127, a = max |y| over the block    (fp32, round to nearest; 0 for a zero block)
+ *   q = clamp(round_half_even(y * (127 / a)), -127, 127)
+ *                                              (int8; the reciprocal and the product rounded
+ *                                               to nearest in fp32; 0 where a = 0)
+ * so y is approximately q * s.  y itself is never written: one pass reads x and writes
+ * the codes and scales.
+ *   x        device bf16 rows, leading dimension ld_x >= d.
+ *   q        device int8 codes, rows of d, leading dimension ld_q >= d.
+ *   scales   device float, rows of d / qblock scales, leading dimension ld_s >= d / qblock.
+ *   qblock   32, 64, 128 or 256, dividing d; else HARP_ERR_INVALID_ARG.
+ * x, q and scales must not overlap.  Runs on the general tiled kernel: radices <= 8,
+ * d % 8 == 0, x and q rows 16-byte aligned (ld_q a multiple of 16), scales 4-byte aligned;
+ * otherwise HARP_ERR_UNSUPPORTED.  rows = 0 is a no-op.  Asynchronous on `stream`.
+ */
+HARP_API harp_status harp_apply_quant(harp_plan_t plan, const void* x, int64_t rows, int64_t ld_x,
+                                      harp_dtype in_dtype, int8_t* q, int64_t ld_q, float* scales,
+                                      int64_t ld_s, int32_t qblock, harp_dir dir, void* stream);
+
+/*
  * harp_apply_columns — every column of an fp32 matrix takes T (FORWARD) or T^T
  * (INVERSE): for j < ncols, y[:, j] = T x[:, j] with x of d = plan dimension rows.  The
  * column side of a two-sided rotation, applied in place without a transpose (HARP

@@ -122,6 +122,37 @@ extern "C" harp_status harp_apply_ex(harp_plan_t p, const void* x, void* y, int6
     return apply_checked(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
 }
 
+extern "C" harp_status harp_apply_quant(harp_plan_t p, const void* x, int64_t rows, int64_t ld_x, harp_dtype in_dtype,
+                                        int8_t* q, int64_t ld_q, float* scales, int64_t ld_s, int32_t qblock,
+                                        harp_dir dir, void* stream) {
+    harp_clear_error();
+    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    if (in_dtype != HARP_BF16) return harp_fail(HARP_ERR_UNSUPPORTED, "the fused quantizer takes bf16 rows");
+    if (dir != HARP_FORWARD && dir != HARP_INVERSE) return harp_fail(HARP_ERR_UNSUPPORTED, "unknown direction");
+    if (rows < 0) return harp_fail(HARP_ERR_INVALID_ARG, "rows < 0");
+    const int64_t d = p->desc.d;
+    if (qblock != 32 && qblock != 64 && qblock != 128 && qblock != 256)
+        return harp_fail(HARP_ERR_INVALID_ARG, "qblock must be 32, 64, 128 or 256");
+    if (d % qblock) return harp_fail(HARP_ERR_INVALID_ARG, "qblock must divide d");
+    if (ld_x < d || ld_q < d || ld_s < d / qblock)
+        return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than the row");
+    if (rows == 0) return HARP_OK;
+    if (!x || !q || !scales) return harp_fail(HARP_ERR_INVALID_ARG, "x, q or scales is NULL");
+    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    harp_status st = check_device(p);
+    if (st != HARP_OK) return st;
+    const size_t xb = ((rows - 1) * ld_x + d) * 2, qb = (rows - 1) * ld_q + d,
+                 sb = ((rows - 1) * ld_s + d / qblock) * sizeof(float);
+    if (ranges_overlap(x, xb, q, qb) || ranges_overlap(x, xb, scales, sb) || ranges_overlap(q, qb, scales, sb))
+        return harp_fail(HARP_ERR_INVALID_ARG, "x, q and scales overlap");
+    QuantOut qo{scales, ld_s, qblock};
+    st = launch_apply_tiled(p, x, q, rows, ld_x, ld_q, HARP_BF16, HARP_BF16, dir, stream, &qo);
+    if (st == HARP_ERR_UNSUPPORTED)
+        return harp_fail(HARP_ERR_UNSUPPORTED, "the fused quantizer needs radices <= 8, d % 8 == 0, 16-byte "
+                                               "aligned x and q rows (ld_q a multiple of 16)");
+    return st;
+}
+
 extern "C" harp_status harp_apply_columns(harp_plan_t p, float* x, int64_t ld_x, int64_t ncols, void* y,
                                           int64_t ld_y, harp_dtype out_dtype, harp_dir dir, void* stream) {
     harp_clear_error();

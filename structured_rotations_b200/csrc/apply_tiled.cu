@@ -57,7 +57,7 @@ int sm_count() {
 
 harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
                                int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
-                               void* stream) {
+                               void* stream, const QuantOut* quant) {
     using namespace harp_tiled;
     const int64_t d = p->desc.d;
     if (d % 8 != 0) return HARP_ERR_UNSUPPORTED;
@@ -67,7 +67,9 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
         mask |= 1 << p->desc.st[t].b;
     }
     if (in_dtype == HARP_F32 && out_dtype == HARP_BF16) return HARP_ERR_UNSUPPORTED;
-    const int64_t es_in = in_dtype == HARP_F32 ? 4 : 2, es_out = out_dtype == HARP_F32 ? 4 : 2;
+    if (quant && in_dtype != HARP_BF16) return HARP_ERR_UNSUPPORTED;
+    const int64_t es_in = in_dtype == HARP_F32 ? 4 : 2;
+    const int64_t es_out = quant ? 1 : out_dtype == HARP_F32 ? 4 : 2;
     if (((uintptr_t)x & 15) || ((uintptr_t)y & 15) || ((ld_x * es_in) & 15) || ((ld_y * es_out) & 15))
         return HARP_ERR_UNSUPPORTED;
     int which = 0;
@@ -109,7 +111,7 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     Shape sh = shape_for(d);
     {
         const char* env = std::getenv("HARP_TILED_SLAB");
-        bool ok = env && !std::strcmp(env, "1") && pd.m >= 2 && pd.st[pd.m - 1].b == 2 && d % 16 == 0 &&
+        bool ok = !quant && env && !std::strcmp(env, "1") && pd.m >= 2 && pd.st[pd.m - 1].b == 2 && d % 16 == 0 &&
                   has_slab_kernel(kMasks[which]) && (pd.st[pd.m - 1].block_off & 3) == 0;
         for (int t = 0; ok && t < pd.m - 1; ++t) ok = ((d / 2) / pd.st[t].b) % 32 == 0;
         if (ok) {
@@ -139,6 +141,9 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
 
     TiledParams tp;
     tp.pd = pd;
+    tp.scales = quant ? quant->scales : nullptr;
+    tp.ld_s = quant ? quant->ld_s : 0;
+    tp.qlanes = quant ? quant->qblock / 8 : 1;
     tp.lanes = p->d_blocks_lanes;
     for (int t = 0; t < HARP_MAX_STAGES; ++t) tp.lane_off[t] = p->lane_off[t];
     tp.x = x;
@@ -168,7 +173,9 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;
     cudaError_t e;
-    if (in_dtype == HARP_BF16 && out_dtype == HARP_BF16)
+    if (quant)
+        e = harp_tiled_launch_bf16_i8(which, V, nt, cl, inv, tp, smem, grid, s);
+    else if (in_dtype == HARP_BF16 && out_dtype == HARP_BF16)
         e = harp_tiled_launch_bf16(which, V, nt, cl, inv, tp, smem, grid, s);
     else if (in_dtype == HARP_F32)
         e = harp_tiled_launch_f32(which, V, nt, cl, inv, tp, smem, grid, s);

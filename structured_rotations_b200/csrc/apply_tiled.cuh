@@ -28,6 +28,8 @@
 // rows (V = 1) with word index i ^ ((i >> 3) & 0x18).
 #pragma once
 
+#include <type_traits>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -66,6 +68,9 @@ struct TiledParams {
     FastDiv nb_div[HARP_MAX_STAGES];   // division by (coordinates per CTA) / b_t
     FastDiv s_div[HARP_MAX_STAGES];    // division by s_t
     const float* last_blocks;          // slab mode: plain 2 x 2 blocks of the last stage
+    float* scales;                     // quantized output (int8 codes in y): per-block scales
+    int64_t ld_s;                      // scales per row of the scales array (row stride)
+    int qlanes;                        // quantizer block / 8: lanes that hold one block
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -442,6 +447,77 @@ __device__ __forceinline__ void drain_tile(const typename VecOf<V>::T* tile, int
     }
 }
 
+// Fused quantizer epilogue (the rotated rows feed a blockwise quantizer, HARP technical
+// summary §2.4: a drop-in preprocessing step in front of the quantizer).  Each aligned
+// block of 8 qlanes coordinates of a row, with maximum magnitude a, becomes one fp32 scale
+// s = a / 127 and int8 codes q = clamp(rne(y * (127 / a)), -127, 127) (the quotient and the
+// reciprocal rounded to nearest in fp32; s = 0 and q = 0 for an all-zero block).  The
+// qlanes consecutive lanes that hold a block, 8 coordinates each, reduce its maximum with
+// shuffles; the NR rows a thread holds reduce in the same shuffle rounds.
+template <int NR>
+__device__ __forceinline__ void quant_rows(const float (&v)[NR][8], int nrows, int8_t* dst, int64_t ld, float* sdst,
+                                           int64_t ld_s, int qlanes, unsigned mask, bool lead) {
+    float a[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        a[r] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[r] = fmaxf(a[r], fabsf(v[r][k]));
+    }
+    for (int o = 1; o < qlanes; o <<= 1) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) a[r] = fmaxf(a[r], __shfl_xor_sync(mask, a[r], o));
+    }
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        if (r >= nrows) break;
+        const float inv = a[r] > 0.f ? __fdiv_rn(127.f, a[r]) : 0.f;
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int q = max(-127, min(127, __float2int_rn(v[r][k] * inv)));
+            w[k >> 2] |= ((uint32_t)q & 0xffu) << (8 * (k & 3));
+        }
+        *(uint2*)(dst + r * ld) = make_uint2(w[0], w[1]);
+        if (lead) sdst[r * ld_s] = __fdiv_rn(a[r], 127.f);
+    }
+}
+
+template <int V, int NT>
+__device__ __forceinline__ void drain_tile_quant(const typename VecOf<V>::T* tile, int d, int nr, int8_t* dst,
+                                                 int64_t ld, int mask, float* sdst, int64_t ld_s, int qlanes) {
+    const int d8 = d / 8;
+    const int lane = threadIdx.x & 31;
+    for (int q = 0; V * q < nr; ++q) {
+        // warp-uniform loop: every lane of a warp takes the same trips, so the shuffles'
+        // mask is exact; lanes past the row's end sit out (whole quantizer blocks)
+        for (int j0 = (int)threadIdx.x - lane; j0 < d8; j0 += NT) {
+            const int j = j0 + lane;
+            const bool act = j < d8;
+            const unsigned amask = __ballot_sync(0xffffffffu, act);
+            if (!act) continue;
+            const bool lead = (j & (qlanes - 1)) == 0;
+            const int sj = j / qlanes;
+            if constexpr (V == 4) {
+                const float4* st = tile + q * d;
+                const int jx = j & 7;
+                float v[4][8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float4 t = st[8 * j + (k ^ jx)];
+                    v[0][k] = t.x, v[1][k] = t.y, v[2][k] = t.z, v[3][k] = t.w;
+                }
+                quant_rows<4>(v, min(4, nr - 4 * q), dst + (4 * q) * ld + 8 * j, ld, sdst + (4 * q) * ld_s + sj,
+                              ld_s, qlanes, amask, lead);
+            } else {
+                float v[1][8];
+                load8(tile + q * d + slot<1>(8 * j, mask), v[0]);
+                quant_rows<1>(v, 1, dst + q * ld + 8 * j, ld, sdst + q * ld_s + sj, ld_s, qlanes, amask, lead);
+            }
+        }
+    }
+}
+
 // CL = 1: one CTA holds whole rows.  CL = 2 (slab mode, schedules whose last radix is 2):
 // a cluster of two CTAs shares each tile, CTA r holding columns [r d/2, (r+1) d/2) of its
 // rows; stages 0..m-2 stay inside a slab, the last one is cross_stage.
@@ -523,7 +599,11 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         } else {
             local_stages(qv);
         }
-        drain_tile<V, NT, TOut>(tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0, p.ld_y, p.mask);
+        if constexpr (std::is_same<TOut, int8_t>::value)
+            drain_tile_quant<V, NT>(tile, dl, nr, (int8_t*)p.y + row0 * p.ld_y, p.ld_y, p.mask,
+                                    p.scales + row0 * p.ld_s, p.ld_s, p.qlanes);
+        else
+            drain_tile<V, NT, TOut>(tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0, p.ld_y, p.mask);
         __syncthreads();
     }
 }
@@ -551,7 +631,7 @@ cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid,
     if constexpr (I < kNumMasks) {
         if (which != I) return launch_mask<TIn, TOut, INV, V, NT, CL, I + 1>(which, tp, smem, grid, stream);
         if constexpr ((V == 1 && !has_row_major_kernel(kMasks[I])) ||
-                      (CL == 2 && (V != 4 || !has_slab_kernel(kMasks[I])))) {
+                      (CL == 2 && (V != 4 || !has_slab_kernel(kMasks[I]) || std::is_same<TOut, int8_t>::value))) {
             return cudaErrorInvalidValue;
         } else {
             auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT, CL>;
@@ -611,3 +691,6 @@ cudaError_t harp_tiled_launch_f32(int which, int V, int nt, int cl, bool inverse
                                   size_t smem, int grid, cudaStream_t stream);
 cudaError_t harp_tiled_launch_bf16_f32(int which, int V, int nt, int cl, bool inverse, const harp_tiled::TiledParams& tp,
                                        size_t smem, int grid, cudaStream_t stream);
+// bf16 rows in, int8 codes and per-block fp32 scales out (the fused quantizer epilogue)
+cudaError_t harp_tiled_launch_bf16_i8(int which, int V, int nt, int cl, bool inverse, const harp_tiled::TiledParams& tp,
+                                      size_t smem, int grid, cudaStream_t stream);

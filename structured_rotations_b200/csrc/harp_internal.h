@@ -96,8 +96,17 @@ harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64
 harp_status launch_cols(const harp_plan_s* p, float* x, int64_t ld_x, int64_t ncols, void* y, int64_t ld_y,
                         harp_dtype out_dtype, harp_dir dir, void* stream);
 
+// Int8 output of the tiled kernel (the fused quantizer epilogue): y receives int8 codes,
+// `scales` one fp32 scale per block of `qblock` coordinates (row stride ld_s floats).
+struct QuantOut {
+    float* scales;
+    int64_t ld_s;
+    int qblock;
+};
+
 // General tiled row kernel (apply_tiled.cu): radices 2..8, d % 8 == 0, 16-byte aligned
 // rows.  Returns HARP_ERR_UNSUPPORTED for other shapes.
 harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
                                int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
-                               void* stream);
+                               void* stream,
+                               const struct QuantOut* quant = nullptr);

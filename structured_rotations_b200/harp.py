@@ -74,6 +74,8 @@ def lib():
         "harp_noalloc_scratch_bytes": (ctypes.c_size_t, []),
         "harp_plan_device_status": (_c_i32, [_vp]),
         "harp_grad_workspace_bytes": (ctypes.c_size_t, [_vp]),
+        "harp_apply_quant": (_c_i32, [_vp, _vp, _c_i64, _c_i64, _c_i32, _vp, _c_i64, _vp, _c_i64, _c_i32, _c_i32,
+                                      _vp]),
         "harp_grad_theta": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _vp, ctypes.c_size_t,
                                      _vp]),
         "harp_plan_destroy": (_c_i32, [_vp]),
@@ -206,6 +208,24 @@ class Plan:
         _check(lib().harp_apply(self._h, x.data_ptr(), y.data_ptr(), n, _ld(x), _ld(y),
                                 _dtype_code(x), d, _stream_handle(stream)), "harp_apply")
         return y
+
+    def apply_quant(self, x, qblock: int = 128, direction: str = "forward", q=None, scales=None, stream=None):
+        """T x (or T^T x) with the fused blockwise quantizer (harp_apply_quant): bf16 rows in,
+        int8 codes [rows, d] and float32 scales [rows, d / qblock] out, y ~= q * scale per
+        aligned block of qblock coordinates.  Returns (q, scales)."""
+        import torch
+        if x.shape[-1] != self.d:
+            raise ValueError(f"last dimension must be d={self.d}")
+        rows = x.shape[0]
+        if q is None:
+            q = torch.empty(rows, self.d, dtype=torch.int8, device=x.device)
+        if scales is None:
+            scales = torch.empty(rows, max(1, self.d // qblock), dtype=torch.float32, device=x.device)
+        d = HARP_FORWARD if direction == "forward" else HARP_INVERSE
+        _check(lib().harp_apply_quant(self._h, x.data_ptr(), rows, _ld(x), _dtype_code(x), q.data_ptr(), _ld(q),
+                                      scales.data_ptr(), _ld(scales), qblock, d, _stream_handle(stream)),
+               "harp_apply_quant")
+        return q, scales
 
     def grad_theta(self, x, g, dtheta=None, workspace=None, stream=None):
         """dL/dtheta for L = sum_r g_r . (T x_r) (harp_grad_theta): the calibration backward
