@@ -468,7 +468,8 @@ def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):
     return {"workload": f"rotate + int8 quantize (qblock {qblock}): d=4096 schedule (8,8,8,8), {w.rows} bf16 rows "
                         f"-> int8 codes + fp32 scales, forward",
             "kernel_ms": ms, "rows_per_s": w.rows / (ms / 1e3), "hbm_gbs": byt / (ms / 1e3) / 1e9,
-            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": H.last_kernel() + " (int8 epilogue)"}
+            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": H.last_kernel() + " (int8 epilogue)",
+            "traffic": recorded_traffic("harp_tiled_kernel", "quant_d4096") if rows is None else None}
 
 
 def grad_roofline(res, clocks, device, torch):
