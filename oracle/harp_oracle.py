@@ -459,3 +459,39 @@ def quantize_blocks(y: np.ndarray, qblock: int):
     safe = np.where(s > 0, s, 1.0)
     q = np.where(s[..., None] > 0, np.rint(yb / safe[..., None]), 0.0)
     return np.clip(q, -127, 127).astype(np.int8).reshape(rows, d), s
+
+
+# ---------------------------------------------------------------------------
+# Composition of rotations
+# ---------------------------------------------------------------------------
+#
+# Composing independent randomized Hadamard transforms brings every input's coordinates
+# close to the behaviour of a uniform random rotation (the RHT-composition results the
+# HARP pages quote: two passes for scalar quantization, three for vector quantization).
+# The composite of plans P_0 .. P_{k-1} is T = T_{k-1} ... T_0 (P_0 acts first); its
+# inverse is T_0^T ... T_{k-1}^T.
+
+class Composed:
+    """T = T_{k-1} ... T_1 T_0 for transforms of one dimension."""
+
+    def __init__(self, transforms: Sequence[Transform]):
+        if not transforms or len({t.plan.d for t in transforms}) != 1:
+            raise ValueError("need transforms of one dimension")
+        self.transforms = list(transforms)
+
+    def forward(self, x: np.ndarray) -> np.ndarray:
+        for t in self.transforms:
+            x = t.forward(x)
+        return x
+
+    def inverse(self, y: np.ndarray) -> np.ndarray:
+        for t in reversed(self.transforms):
+            y = t.inverse(y)
+        return y
+
+    def apply(self, x: np.ndarray, direction: str) -> np.ndarray:
+        if direction == "forward":
+            return self.forward(x)
+        if direction == "inverse":
+            return self.inverse(x)
+        raise ValueError(direction)
