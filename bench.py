@@ -440,7 +440,42 @@ def side_measurements(args, H, W, torch, device, peak):
                 "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
     del wt, wo, ws
     out.append(quant_measurement(args, H, W, torch, device, peak))
+    out.append(compose_measurement(args, H, W, torch, device, peak))
     return out
+
+
+def compose_measurement(args, H, W, torch, device, peak):
+    """Two rotations composed (harp_plan_compose) on the d = 4096 workload's rows: the C2
+    plan, then a second (8,8,8,8) plan (theta seed + 1, sign seed + 1), in one pass; beside
+    it the same two plans as two separate passes with a bf16 intermediate."""
+    w = W.get("d4096")
+    p1 = make_plan("d4096", H, W)
+    th2 = W.draw_theta(H.theta_count(w.schedule), w.theta_sigma, w.theta_seed + 1)
+    p2 = H.Plan(w.d, w.schedule, theta=th2, sign_seed=w.sign_seed + 1).materialize()
+    comp = H.Plan.compose([p1, p2])
+    x = to_device_bf16(W.draw_encoded(w, 0, w.rows), torch, device)
+    y = torch.empty_like(x)
+    st = max(3, args.steps // 4)
+    el, km, _, kn = time_apply(comp, x, y, st, 3, torch)
+    mid = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        p1.apply(x, mid)
+        p2.apply(mid, y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(st):
+        p1.apply(x, mid)
+        p2.apply(mid, y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    two = e0.elapsed_time(e1) / st
+    byt = 2 * w.rows * w.d * 2
+    return {"workload": "two rotations composed: d=4096 (8,8,8,8) x 2, 65536 bf16 rows, one pass",
+            "kernel_ms": km, "rows_per_s": w.rows / (km / 1e3), "hbm_gbs": byt / (km / 1e3) / 1e9,
+            "hbm_frac": byt / (km / 1e3) / 1e9 / peak, "kernel": kn,
+            "two_passes_ms": two, "two_passes_kernels": "harp_fast_d4096_fwd_kernel x 2 (bf16 between)"}
 
 
 def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):

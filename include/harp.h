@@ -288,6 +288,22 @@ HARP_API harp_status harp_grad_theta(harp_plan_t plan, const void* x, const void
                                      int64_t ld_x, int64_t ld_g, harp_dtype dtype, float* dtheta,
                                      void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * harp_plan_compose — one plan for the composition T = T_{k-1} ... T_1 T_0 of k plans of
+ * the same dimension (plans[0] acts first): k independent rotations in one pass over the
+ * rows (composing two or three randomized Hadamard transforms brings every input's
+ * coordinates close to the behaviour of a uniform random rotation, the RHT-composition
+ * results the HARP pages quote).  The composite copies the plans' device blocks (the
+ * plans may be destroyed afterwards) and is materialized on the current device; every
+ * plan must be materialized there, and the stages must number at most HARP_MAX_STAGES in
+ * all (HARP_ERR_SCHEDULE otherwise).  The composite works with harp_apply, harp_apply_ex,
+ * harp_apply_host, harp_apply_quant (INVERSE gives T^T = T_0^T ... T_{k-1}^T) and as a side
+ * of harp_apply_two_sided; harp_apply_columns, harp_grad_theta, harp_plan_signs and
+ * harp_plan_base_mixer return HARP_ERR_UNSUPPORTED for it.  Destroy with
+ * harp_plan_destroy.  Asynchronous copies on `stream`.
+ */
+HARP_API harp_status harp_plan_compose(harp_plan_t* out, const harp_plan_t* plans, int32_t k, void* stream);
+
 /* harp_plan_device_status — synchronizes the plan's device and reports whether any
  * bounded device-side wait of a kernel launched with this plan gave up since the
  * last call: HARP_ERR_TIMEOUT if one did (the flag is then cleared), HARP_OK if

@@ -111,7 +111,7 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     Shape sh = shape_for(d);
     {
         const char* env = std::getenv("HARP_TILED_SLAB");
-        bool ok = !quant && env && !std::strcmp(env, "1") && pd.m >= 2 && pd.st[pd.m - 1].b == 2 && d % 16 == 0 &&
+        bool ok = !quant && !p->composite && env && !std::strcmp(env, "1") && pd.m >= 2 && pd.st[pd.m - 1].b == 2 && d % 16 == 0 &&
                   has_slab_kernel(kMasks[which]) && (pd.st[pd.m - 1].block_off & 3) == 0;
         for (int t = 0; ok && t < pd.m - 1; ++t) ok = ((d / 2) / pd.st[t].b) % 32 == 0;
         if (ok) {

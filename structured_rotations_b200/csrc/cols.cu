@@ -244,6 +244,7 @@ harp_status launch_cols(const harp_plan_s* pl, float* x, int64_t ld_x, int64_t n
                         harp_dtype out_dtype, harp_dir dir, void* stream_) {
     const PlanDesc& pd = pl->desc;
     const int64_t d = pd.d;
+    if (pl->composite) return HARP_ERR_UNSUPPORTED;   // the split below needs s_t = prod_{j<t} b_j
     if (pd.m < 2 || ncols <= 0 || ncols > (int64_t)1 << 30) return HARP_ERR_UNSUPPORTED;
     for (int t = 0; t < pd.m; ++t)
         if (pd.st[t].b > 8) return HARP_ERR_UNSUPPORTED;

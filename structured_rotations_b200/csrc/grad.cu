@@ -409,6 +409,7 @@ extern "C" harp_status harp_grad_theta(harp_plan_t p, const void* x, const void*
     const int64_t d = pd.d;
     if (ld_x < d || ld_g < d) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than d");
     if (!dtheta) return harp_fail(HARP_ERR_INVALID_ARG, "dtheta is NULL");
+    if (p->composite) return harp_fail(HARP_ERR_UNSUPPORTED, "the gradient is taken for one plan, not a composite");
     if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -47,6 +47,7 @@ struct harp_plan_s {
     // device side (owned)
     int device = -1;
     bool materialized = false;
+    bool composite = false;           // built by harp_plan_compose: stages of several plans in a row
     float* d_blocks = nullptr;        // signed blocks, [stage][c][k][l]
     float* d_blocks_lanes = nullptr;  // the same, lane-interleaved (see lane_off)
     void* d_theta = nullptr;          // float or int8 codes, as stored

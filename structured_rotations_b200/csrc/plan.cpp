@@ -242,6 +242,7 @@ harp_status harp_plan_destroy(harp_plan_t plan) {
 
 harp_status harp_plan_base_mixer(harp_plan_t plan, int32_t radix, double* out) {
     if (!plan || !out) return harp_fail(HARP_ERR_INVALID_ARG, "NULL argument");
+    if (plan->composite) return harp_fail(HARP_ERR_UNSUPPORTED, "a composite has the mixers of its plans");
     auto it = plan->mixer_index.find(radix);
     if (it == plan->mixer_index.end()) return harp_fail(HARP_ERR_INVALID_ARG, "radix not in the plan");
     std::memcpy(out, plan->mixers.data() + it->second, sizeof(double) * radix * radix);
@@ -250,6 +251,7 @@ harp_status harp_plan_base_mixer(harp_plan_t plan, int32_t radix, double* out) {
 
 harp_status harp_plan_signs(harp_plan_t plan, int8_t* out) {
     if (!plan || !out) return harp_fail(HARP_ERR_INVALID_ARG, "NULL argument");
+    if (plan->composite) return harp_fail(HARP_ERR_UNSUPPORTED, "a composite has the signs of its plans");
     std::memcpy(out, plan->signs.data(), plan->signs.size());
     return HARP_OK;
 }

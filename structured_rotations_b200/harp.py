@@ -74,6 +74,7 @@ def lib():
         "harp_noalloc_scratch_bytes": (ctypes.c_size_t, []),
         "harp_plan_device_status": (_c_i32, [_vp]),
         "harp_grad_workspace_bytes": (ctypes.c_size_t, [_vp]),
+        "harp_plan_compose": (_c_i32, [ctypes.POINTER(_vp), ctypes.POINTER(_vp), _c_i32, _vp]),
         "harp_apply_quant": (_c_i32, [_vp, _vp, _c_i64, _c_i64, _c_i32, _vp, _c_i64, _vp, _c_i64, _c_i32, _c_i32,
                                       _vp]),
         "harp_grad_theta": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _vp, ctypes.c_size_t,
@@ -189,6 +190,23 @@ class Plan:
     @property
     def handle(self):
         return self._h
+
+    @classmethod
+    def compose(cls, plans: Sequence["Plan"], stream=None) -> "Plan":
+        """One plan for T_{k-1} ... T_0 of materialized plans of one dimension (plans[0]
+        acts first), applied in a single pass (harp_plan_compose)."""
+        if not plans:
+            raise ValueError("need at least one plan")
+        arr = (_vp * len(plans))(*[p.handle for p in plans])
+        handle = _vp()
+        _check(lib().harp_plan_compose(ctypes.byref(handle), arr, len(plans), _stream_handle(stream)),
+               "harp_plan_compose")
+        c = cls.__new__(cls)
+        c.d = plans[0].d
+        c.schedule = tuple(b for p in plans for b in p.schedule)
+        c._keep = ()
+        c._h = handle
+        return c
 
     def materialize(self, stream=None) -> "Plan":
         _check(lib().harp_materialize_blocks(self._h, _stream_handle(stream)), "harp_materialize_blocks")
