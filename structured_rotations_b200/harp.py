@@ -206,6 +206,7 @@ class Plan:
         c.schedule = tuple(b for p in plans for b in p.schedule)
         c._keep = ()
         c._h = handle
+        c.composite = True
         return c
 
     def materialize(self, stream=None) -> "Plan":
@@ -253,7 +254,9 @@ class Plan:
         import torch
         if x.dtype != g.dtype or x.shape != g.shape or x.shape[-1] != self.d:
             raise ValueError(f"x and g must be rows of d={self.d} of one dtype")
-        n = theta_count(self.schedule)
+        # a composite's schedule is its plans' schedules in a row (no theta count of its
+        # own): the library declines it, so any buffer does
+        n = theta_count(self.schedule) if not getattr(self, "composite", False) else 1
         if dtheta is None:
             dtheta = torch.empty(n, dtype=torch.float32, device=x.device)
         if dtheta.dtype != torch.float32 or dtheta.numel() != n or not dtheta.is_contiguous():
