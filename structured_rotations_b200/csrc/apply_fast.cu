@@ -64,7 +64,6 @@ struct FastParams {
     int ntiles;
     const float4* frag;      // B fragments, [cta rank][warp][column / 4][lane] float4 (see pack kernel)
     int* status;
-    float zero;              // 0.0f, passed at run time (see split2_tf32)
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -73,25 +72,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// Two values split at once into x = hi + lo with packed fp32 arithmetic (Veltkamp's
-// splitting with factor 2^13 + 1): t = 8193 x rounded, hi = t - (t - x) has 11
-// significant bits, so it is exact in TF32, and lo = x - hi is exact in fp32; the tensor
-// core reads the top 19 bits of lo, so |x - hi - lo_tf32| <= 2^-22 |x|.  All four
-// operations are round-to-nearest f32x2 instructions on the FMA pipe.  t is formed as
-// an FMA with a zero addend that only the caller knows (`zero2`), so the compiler cannot
-// contract the product into the subtractions, which would make hi == x.
-// Valid for |x| < 2^115.
-__device__ __forceinline__ void split2_tf32(float a, float b, unsigned long long zero2, uint32_t& ha,
-                                            uint32_t& hb, uint32_t& la, uint32_t& lb) {
-    unsigned long long x, c, t, d, hi, lo;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a), "f"(b));
-    asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(8193.0f));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(x), "l"(c), "l"(zero2));
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(t), "l"(x));
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(hi) : "l"(t), "l"(d));
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(lo) : "l"(x), "l"(hi));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(ha), "=r"(hb) : "l"(hi));
-    asm("mov.b64 {%0, %1}, %2;" : "=r"(la), "=r"(lb) : "l"(lo));
+// Two values split into x = hi + lo for the three-product TF32 scheme.  hi is x rounded to
+// 11 significant bits (ties away from zero) by integer arithmetic on its bit pattern: add
+// half of bit 13, clear bits 0-12 (a carry into the exponent is the correct rounding), so
+// hi is exact in TF32; lo = x - hi is exact in fp32 (at most 13 significant bits), and the
+// tensor core reads its top 11, so |x - hi - lo_tf32| <= 2^-22 |x|.  The rounding runs on
+// the integer ALU pipe and only the subtraction on the FMA pipe, which the tensor-core
+// stages keep busy otherwise.  Valid for finite x below the largest binade.
+__device__ __forceinline__ void split2_tf32(float a, float b, uint32_t& ha, uint32_t& hb, uint32_t& la,
+                                            uint32_t& lb) {
+    ha = (__float_as_uint(a) + 0x1000u) & 0xffffe000u;
+    hb = (__float_as_uint(b) + 0x1000u) & 0xffffe000u;
+    la = __float_as_uint(__fsub_rn(a, __uint_as_float(ha)));
+    lb = __float_as_uint(__fsub_rn(b, __uint_as_float(hb)));
 }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -263,14 +256,14 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // A fragments split into hi + lo and the B fragments (two fp32 words per group, from
 // TMEM) split likewise; three products per group.
 __device__ __forceinline__ void mma_stage_f32(const float (&a)[8][4], const uint32_t (&bw)[16],
-                                              unsigned long long z2, float (&d)[8][4]) {
+                                              float (&d)[8][4]) {
 #pragma unroll
     for (int l = 0; l < 8; ++l) {
         uint32_t ah[4], al[4];
-        split2_tf32(a[l][0], a[l][1], z2, ah[0], ah[1], al[0], al[1]);
-        split2_tf32(a[l][2], a[l][3], z2, ah[2], ah[3], al[2], al[3]);
+        split2_tf32(a[l][0], a[l][1], ah[0], ah[1], al[0], al[1]);
+        split2_tf32(a[l][2], a[l][3], ah[2], ah[3], al[2], al[3]);
         uint32_t bh0, bl0, bh1, bl1;
-        split2_tf32(__uint_as_float(bw[2 * l]), __uint_as_float(bw[2 * l + 1]), z2, bh0, bh1, bl0, bl1);
+        split2_tf32(__uint_as_float(bw[2 * l]), __uint_as_float(bw[2 * l + 1]), bh0, bh1, bl0, bl1);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         mma_tf32(acc, ah, bh0, bh1);
         mma_tf32(acc, ah, bl0, bl1);
@@ -378,8 +371,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int r = (int)cluster_rank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     unsigned char* Xw = X + warp * kXBytes;
-    unsigned long long z2;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(z2) : "f"(p.zero));
 
     // tensor memory: the whole 512 columns; warp w uses lanes 32 (w & 3).., columns 128 (w >> 2)..
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
@@ -448,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 8; ++j) {
                 const uint32_t a[4] = {w0[j] << 16, w1[j] << 16, w0[j] & 0xffff0000u, w1[j] & 0xffff0000u};
                 uint32_t bh0, bl0, bh1, bl1;
-                split2_tf32(__uint_as_float(bw[2 * j]), __uint_as_float(bw[2 * j + 1]), z2, bh0, bh1, bl0, bl1);
+                split2_tf32(__uint_as_float(bw[2 * j]), __uint_as_float(bw[2 * j + 1]), bh0, bh1, bl0, bl1);
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_tf32(d, a, bh0, bh1);
                 mma_tf32(d, a, bl0, bl1);
@@ -473,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // stage 1: group l = i0; output slot 2q <-> i1 = q (pencils of CTA 0),
             // 2q+1 <-> i1 = q + 4 (pencils of CTA 1); both are pencil a_local = l + 8q there.
             float y1[8][4];
-            mma_stage_f32(a1, bw, z2, y1);
+            mma_stage_f32(a1, bw, y1);
             if (task == 0) {
                 // row `warp` of the previous tile's output leaves O, which aliases the part
                 // of S this warp is about to write
@@ -531,14 +522,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             tmem_wait_ld();
             float zz2[8][4];
-            mma_stage_f32(v2, bw, z2, zz2);
+            mma_stage_f32(v2, bw, zz2);
             tmem_ld16(taddr + 32u * (2 + task) + 16u, bw);   // stage-3 fragments
             float a3[8][4];
             quad_butterfly(zz2, q, a3);
             tmem_wait_ld();
             // stage 3: group l = i2; output slot 2q <-> i3 = 2q, 2q+1 <-> i3 = 2q + 1
             float y3[8][4];
-            mma_stage_f32(a3, bw, z2, y3);
+            mma_stage_f32(a3, bw, y3);
             if (task == 0) cluster_wait();   // my copies have landed too: O (= S) may be written
             // bf16 runs of 8 consecutive beta (i2 = 0..7) for i3 = 2q + e, rows g and g + 8
 #pragma unroll
@@ -698,7 +689,6 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     fp.ntiles = (int)ntiles;
     fp.frag = reinterpret_cast<const float4*>(fs->frag);
     fp.status = p->d_status;
-    fp.zero = 0.0f;
     harp_fast_d4096_fwd_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
