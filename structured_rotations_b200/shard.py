@@ -92,3 +92,18 @@ def two_sided_row_sharded(plan_u, plan_v, w_local, group=None, *, work_dtype=Non
     else:
         back.copy_(res.view(world, n_local, c))
     return back.transpose(0, 1).reshape(n_local, n_in)
+
+
+def grad_theta_sharded(plan, x_local, g_local, group=None, *, grad_fn=None):
+    """dL/dtheta for L = sum_r g_r . (T x_r) over the rows of every rank of `group`, each rank
+    holding its own rows x_local and upstream gradients g_local (HARP technical summary §2.3:
+    theta is fitted from calibration data, spread here over the ranks).  Each rank forms the
+    gradient of its rows (harp_grad_theta), then one all-reduce sums them, so every rank
+    ends with the same dL/dtheta.  `grad_fn(x, g)` replaces the library call (tests run the
+    exchange on CPU ranks with a float64 reference in its place)."""
+    import torch.distributed as dist
+
+    d = plan.grad_theta(x_local, g_local) if grad_fn is None else grad_fn(x_local, g_local)
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(d, op=dist.ReduceOp.SUM, group=group)
+    return d

@@ -123,3 +123,69 @@ def test_two_sided_workspace_bytes():
 
 def test_destroy_null_is_ok():
     assert H.lib().harp_plan_destroy(None) == HB.HARP_OK
+
+
+@pytest.mark.parametrize("schedule", [(8, 8), (8, 8, 8, 5, 2), (3, 5, 7), (2,) * 6])
+def test_grad_workspace_bytes(schedule):
+    # one float per block entry, each stage padded to a multiple of 4 floats (16 bytes)
+    d = int(np.prod(schedule))
+    plan = H.Plan(d, schedule)
+    want = sum(((d // b) * b * b + 3) // 4 * 4 for b in schedule) * 4
+    assert H.lib().harp_grad_workspace_bytes(plan.handle) == want
+    assert H.lib().harp_grad_workspace_bytes(None) == 0
+
+
+def test_grad_theta_argument_errors_before_any_device_call():
+    L = H.lib()
+    plan = H.Plan(64, (8, 8))
+    p = ctypes.c_void_p(16)
+    ws = int(L.harp_grad_workspace_bytes(plan.handle))
+    args = lambda **kw: dict(dict(plan=plan.handle, x=p, g=p, rows=4, ld_x=64, ld_g=64, dtype=HB.HARP_F32,
+                                  dtheta=p, ws=p, ws_bytes=ws, stream=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.harp_grad_theta(a["plan"], a["x"], a["g"], a["rows"], a["ld_x"], a["ld_g"], a["dtype"],
+                                 a["dtheta"], a["ws"], a["ws_bytes"], a["stream"])
+
+    assert call(plan=None) == HB.HARP_ERR_INVALID_ARG
+    assert call(dtype=7) == HB.HARP_ERR_UNSUPPORTED
+    assert call(rows=-1) == HB.HARP_ERR_INVALID_ARG
+    assert call(ld_g=63) == HB.HARP_ERR_INVALID_ARG
+    assert call(dtheta=None) == HB.HARP_ERR_INVALID_ARG
+    assert call() == HB.HARP_ERR_NOT_MATERIALIZED
+
+
+def test_apply_quant_argument_errors_before_any_device_call():
+    L = H.lib()
+    plan = H.Plan(4096, (8, 8, 8, 8))
+    p = ctypes.c_void_p(16)
+
+    def call(plan_h=plan.handle, x=p, rows=4, ld_x=4096, dtype=HB.HARP_BF16, q=p, ld_q=4096, s=p, ld_s=32,
+             qblock=128, direction=HB.HARP_FORWARD):
+        return L.harp_apply_quant(plan_h, x, rows, ld_x, dtype, q, ld_q, s, ld_s, qblock, direction, None)
+
+    assert call(plan_h=None) == HB.HARP_ERR_INVALID_ARG
+    assert call(dtype=HB.HARP_F32) == HB.HARP_ERR_UNSUPPORTED
+    assert call(direction=5) == HB.HARP_ERR_UNSUPPORTED
+    assert call(rows=-1) == HB.HARP_ERR_INVALID_ARG
+    for qb in (16, 48, 512):
+        assert call(qblock=qb) == HB.HARP_ERR_INVALID_ARG
+    assert call(ld_q=4095) == HB.HARP_ERR_INVALID_ARG
+    assert call(qblock=256, ld_s=15) == HB.HARP_ERR_INVALID_ARG
+    assert call(rows=0, x=None, q=None, s=None) == HB.HARP_OK
+    assert call(q=None) == HB.HARP_ERR_INVALID_ARG
+    assert call() == HB.HARP_ERR_NOT_MATERIALIZED
+    odd = H.Plan(96, (8, 4, 3))                                         # 64 does not divide 96
+    assert call(plan_h=odd.handle, ld_x=96, ld_q=96, ld_s=2, qblock=64) == HB.HARP_ERR_INVALID_ARG
+
+
+def test_plan_compose_argument_errors_before_any_device_call():
+    L = H.lib()
+    out = ctypes.c_void_p()
+    keep = H.Plan(64, (8, 8))
+    plans = (ctypes.c_void_p * 1)(keep.handle)
+    assert L.harp_plan_compose(None, plans, 1, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_plan_compose(ctypes.byref(out), plans, 0, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_plan_compose(ctypes.byref(out), None, 1, None) == HB.HARP_ERR_INVALID_ARG
+    assert not out.value

@@ -154,3 +154,48 @@ def test_two_sided_row_sharded_exchange(tmp_path, world):
     r = json.load(open(tmp_path / "two_sided.json"))
     assert r["shape"] == [64, 16]
     assert r["max_err"] < 1e-12
+
+
+def _grad_worker(rank, world, port, out_dir):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import workloads as W
+    from oracle import harp_oracle as O
+    from structured_rotations_b200.shard import grad_theta_sharded, strong_shard
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        sched = (8, 2, 4)
+        plan = O.make_plan(64, sched, W.draw_theta(O.theta_count(sched), 0.3, 3), sign_seed=4)
+        rng = np.random.default_rng(21)
+        x, g = rng.standard_normal((37, 64)), rng.standard_normal((37, 64))
+        r0, n = strong_shard(37, world, rank)
+
+        def grad_fn(xl, gl):
+            return torch.from_numpy(O.theta_grad(plan, xl.numpy(), gl.numpy()))
+
+        got = grad_theta_sharded(None, torch.from_numpy(x[r0:r0 + n].copy()), torch.from_numpy(g[r0:r0 + n].copy()),
+                                 grad_fn=grad_fn)
+        parts = [None] * world
+        dist.all_gather_object(parts, got.numpy())
+        if rank == 0:
+            want = O.theta_grad(plan, x, g)
+            with open(os.path.join(out_dir, "grad.json"), "w") as f:
+                json.dump({"max_err": float(max(np.abs(p_ - want).max() for p_ in parts)),
+                           "scale": float(np.abs(want).max())}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_grad_theta_sharded_sums_over_ranks(tmp_path, world):
+    """The calibration backward over row shards (each rank its rows' gradient, one
+    all-reduce) gives every rank the gradient of all rows, on gloo ranks with a float64
+    reference as each rank's compute."""
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.spawn(_grad_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    r = json.load(open(tmp_path / "grad.json"))
+    assert r["max_err"] <= 1e-12 * max(1.0, r["scale"])
