@@ -47,6 +47,14 @@ statistics, scipy's Sylvester Hadamard, the unique positive-diagonal QR, Givens
 group law, Cayley orthogonality / det +1 / closed forms, theta=0 Kronecker form,
 an independent tensor-axis restatement of the stages, dense orthogonality,
 round trips and bf16 rounding of hand-worked values.
+
+Beyond the forward transform, three parts that build on it (each with its own pins):
+the calibration backward dL/dtheta (§2.3; tests/test_oracle_grad_pins.py: central
+differences, one-stage closed forms, stationarity, additivity), the blockwise int8
+quantizer of the rotated rows (§2.4; tests/test_oracle_quant_pins.py: hand-worked
+codes, zero blocks, the half-step bound, scaling) and the composition of rotations
+(tests/test_oracle_compose_pins.py: the theta = 0 product of signed Hadamards,
+orthogonality, inverse, factor order).
 """
 from __future__ import annotations
 
