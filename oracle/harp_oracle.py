@@ -503,3 +503,49 @@ class Composed:
         if direction == "inverse":
             return self.inverse(x)
         raise ValueError(direction)
+
+
+# ---------------------------------------------------------------------------
+# The fit's evaluation terms on a Hessian proxy (§2.3 Optimization Objective)
+# ---------------------------------------------------------------------------
+#
+# The pages describe the two terms of L_fit = L_diag + lambda_bd R_bd in words only; the
+# readings here:
+#  * the input-side Hessian proxy H (d_in x d_in, symmetric positive definite, e.g. X^T X of
+#    calibration activations) in the rotated basis: inputs rotate as x' = T_V^T x, so
+#    H' = T_V^T H T_V;
+#  * R_bd: the energy of H' outside the diagonal blocks of the quantizer's block size q,
+#    as a fraction of its total energy, sum_{I != J} |H'_IJ|_F^2 / |H'|_F^2;
+#  * L_diag: the rotated weight W' = T_U^T W T_V against its blockwise target Q(W')
+#    (the round-to-nearest int8 quantizer of quantize_blocks along the rows, dequantized),
+#    each column j weighted by the diagonal of H': sum_j H'_jj sum_r (W'_rj - Q(W')_rj)^2.
+
+def rotated_hessian(plan_v: OraclePlan, h: np.ndarray) -> np.ndarray:
+    """H' = T_V^T H T_V."""
+    tv = Transform(plan_v)
+    z = tv.inverse(np.asarray(h, dtype=np.float64))      # rows: (T_V^T h_r)^T = h_r^T T_V
+    return tv.inverse(z.T).T                             # columns: T_V^T (H T_V)
+
+
+def off_block_energy(h: np.ndarray, q: int) -> float:
+    """sum over blocks I != J of |H_IJ|_F^2 over |H|_F^2, blocks of q x q."""
+    h = np.asarray(h, dtype=np.float64)
+    n = h.shape[0]
+    if h.shape != (n, n) or n % q:
+        raise ValueError("square matrix with q dividing its size")
+    total = float(np.sum(h * h))
+    blk = np.arange(n) // q
+    off = float(np.sum((h * h)[blk[:, None] != blk[None, :]]))   # summed directly, not total - diag
+    return off / total if total > 0 else 0.0
+
+
+def r_bd(plan_v: OraclePlan, h: np.ndarray, q: int) -> float:
+    return off_block_energy(rotated_hessian(plan_v, h), q)
+
+
+def l_diag(w_rot: np.ndarray, h_rot: np.ndarray, q: int) -> float:
+    """sum_j H'_jj sum_r (W'_rj - Q(W')_rj)^2 for the rotated weight and Hessian proxy."""
+    w = np.asarray(w_rot, dtype=np.float64)
+    codes, scales = quantize_blocks(w, q)
+    target = (codes.reshape(w.shape[0], -1, q) * scales[..., None]).reshape(w.shape)
+    return float(np.sum(np.diag(h_rot)[None, :] * (w - target) ** 2))
