@@ -134,6 +134,10 @@ HARP_API harp_status harp_materialize_blocks(harp_plan_t plan, void* stream);
  * multiply-adds (the specialized d = 4096 kernel forms the products on tensor cores from
  * TF32 hi/lo splits of both operands, three passes, fp32 accumulation), the output
  * rounded to `dtype` to nearest even.
+ * Ordering: the first call that takes the specialized d = 4096 kernel for a plan (bf16,
+ * FORWARD, 32 rows or more) builds that kernel's coefficient table on its stream; calls on
+ * other streams must be ordered after that first call (an event or a synchronize), and
+ * that first call must not run concurrently with another call on the same plan.
  */
 HARP_API harp_status harp_apply(harp_plan_t plan, const void* x, void* y, int64_t rows,
                        int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
@@ -155,7 +159,8 @@ HARP_API harp_status harp_apply_ex(harp_plan_t plan, const void* x, void* y, int
  * kernels and device-to-host copies overlap (page-locked host memory is needed for the
  * overlap; pageable memory works, the copies then serialize).  Synchronous: returns when y
  * holds the result.  Runs on the current device, which must be the plan's.  The plan keeps
- * the streams and six device buffers of one chunk until harp_plan_destroy.
+ * the streams and six device buffers of one chunk until harp_plan_destroy; calls on one
+ * plan from several host threads take turns (a lock of the plan's).
  *   x, y        host pointers, element type dtype; y may equal x (then ld_x == ld_y); any
  *               other overlap returns HARP_ERR_INVALID_ARG.
  *   rows, ld_x, ld_y, dtype, dir   as harp_apply.

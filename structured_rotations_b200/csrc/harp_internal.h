@@ -3,6 +3,7 @@
 
 #include <cstdint>
 #include <map>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -57,6 +58,7 @@ struct harp_plan_s {
     int* d_status = nullptr;          // device error word (bounded waits)
     void* fast = nullptr;             // fast-path state (see apply_fast.cu)
     void* host_io = nullptr;          // streams and staging buffers of harp_apply_host (host_io.cu)
+    std::mutex host_io_mu;            // harp_apply_host calls on this plan take turns
 };
 
 // error reporting (plan.cpp)

@@ -4,6 +4,7 @@
 // and its device-to-host copy follow each other in order, and the three streams overlap,
 // so the two copy directions (separate copy engines) and the kernels run at once.
 #include <algorithm>
+#include <mutex>
 
 #include <cuda_runtime.h>
 
@@ -105,6 +106,7 @@ extern "C" harp_status harp_apply_host(harp_plan_t p, const void* x, void* y, in
         return harp_fail(HARP_ERR_INVALID_ARG, "in-place apply needs ld_x == ld_y");
     }
     const int64_t chunk = std::max<int64_t>(32, std::min<int64_t>(rows, (int64_t)(kChunkBytes / row_bytes)));
+    std::lock_guard<std::mutex> lock(p->host_io_mu);   // the plan's streams and buffers serve one call at a time
     harp_status st = ensure(p, (size_t)chunk * row_bytes);
     if (st != HARP_OK) return st;
     HostIo* h = (HostIo*)p->host_io;
