@@ -199,3 +199,15 @@ def test_grad_theta_sharded_sums_over_ranks(tmp_path, world):
     mp.spawn(_grad_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True)
     r = json.load(open(tmp_path / "grad.json"))
     assert r["max_err"] <= 1e-12 * max(1.0, r["scale"])
+
+
+def test_grad_theta_sharded_without_a_process_group_is_the_local_gradient():
+    import torch
+    from structured_rotations_b200.shard import grad_theta_sharded
+
+    class FakePlan:
+        def grad_theta(self, x, g):
+            return (x * g).sum(dim=0)
+
+    x, g = torch.arange(12.0).reshape(3, 4), torch.ones(3, 4)
+    assert torch.equal(grad_theta_sharded(FakePlan(), x, g), (x * g).sum(dim=0))
