@@ -305,7 +305,8 @@ HARP_API harp_status harp_grad_theta(harp_plan_t plan, const void* x, const void
  * harp_apply_host, harp_apply_quant (INVERSE gives T^T = T_0^T ... T_{k-1}^T) and as a side
  * of harp_apply_two_sided; harp_apply_columns, harp_grad_theta, harp_plan_signs and
  * harp_plan_base_mixer return HARP_ERR_UNSUPPORTED for it.  Destroy with
- * harp_plan_destroy.  Asynchronous copies on `stream`.
+ * harp_plan_destroy.  The copies run on `stream` and the call returns when they are done
+ * (not allowed inside a stream capture).
  */
 HARP_API harp_status harp_plan_compose(harp_plan_t* out, const harp_plan_t* plans, int32_t k, void* stream);
 

@@ -85,6 +85,8 @@ extern "C" harp_status harp_plan_compose(harp_plan_t* out, const harp_plan_t* pl
         boff += p->block_floats;
         loff += p->lane_floats;
     }
+    // wait for the copies, so that the source plans may be destroyed as soon as this returns
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     c->materialized = true;
     *out = c;
