@@ -266,11 +266,24 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "rows_per_step": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{sample} rows of the workload per step (float64 scipy CSR stages, one core)"},
+                         "host_cores": host_threads()[0], "thread_env": host_threads()[1],
+                         "sample": f"{sample} rows of the workload per step (float64 scipy CSR stages, one core "
+                                   f"of {host_threads()[0]})"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
     return 0
+
+
+def host_threads():
+    """The host's usable cores and the BLAS / OpenMP thread settings, recorded beside the
+    oracle's timing (its scipy CSR stage products run on one core)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    env = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    return cores, {k: v for k, v in env.items() if v is not None}
 
 
 def cpu_baseline(args, W):
@@ -285,9 +298,11 @@ def cpu_baseline(args, W):
         tr.forward(x)
         rows += chunk
     dt = time.perf_counter() - t0
+    host_cores, blas_env = host_threads()
     return {"value": rows / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "host_cores": host_cores, "thread_env": blas_env,
             "sample": f"{rows} rows of the workload ({chunk}-row chunks, float64 scipy CSR stages, "
-                      f"one core) in {dt:.1f} s"}
+                      f"one core of {host_cores}) in {dt:.1f} s"}
 
 
 # ------------------------------------------------------------------ ours ---
@@ -408,10 +423,14 @@ def side_measurements(args, H, W, torch, device, peak):
         yd = torch.empty_like(xd)
         for direction in ("forward", "inverse"):
             dev_us, host_us, wall_us, kn = time_calls(pd_, xd, yd, 200, 20, torch, direction)
+            coef = 4 * wd.d * sum(wd.schedule)      # the plan's fp32 blocks, read once per call
+            rb = 4 * rows_d * wd.d
             out.append({"workload": f"d=8192 schedule (8,8,8,8,2), int8 theta, {rows_d} bf16 rows (decode-shaped), "
                                     f"{direction}", "rows_per_s": rows_d / (wall_us / 1e6),
                         "us_per_call": wall_us, "device_us_per_call": dev_us, "host_us_per_call": host_us,
-                        "kernel": kn, "hbm_frac": 4 * rows_d * wd.d / (dev_us / 1e6) / 1e9 / peak})
+                        "kernel": kn, "row_bytes": rb, "coefficient_bytes": coef,
+                        "row_hbm_frac": rb / (dev_us / 1e6) / 1e9 / peak,
+                        "hbm_frac": (rb + coef) / (dev_us / 1e6) / 1e9 / peak})
         del xd, yd
     del pd_
     # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)
@@ -438,10 +457,54 @@ def side_measurements(args, H, W, torch, device, peak):
     b4 = 2 * (2 * w4.n_out * w4.n_in * 2)        # two passes, each reading and writing W once
     out.append({"workload": WORKLOAD_TEXT["two_sided"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
                 "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
+    out.append(fit_measurement(H, W, torch, device, peak, pv, wo, w4))
     del wt, wo, ws
     out.append(quant_measurement(args, H, W, torch, device, peak))
     out.append(compose_measurement(args, H, W, torch, device, peak))
     return out
+
+
+def fit_measurement(H, W, torch, device, peak, pv, w_rot, w4, q=128, steps=10):
+    """The fit's evaluation terms on the two-sided workload's shapes: the Hessian proxy of
+    the V side (8192 x 8192, fp32) rotated to H' = T_V^T H T_V by the two-sided rotation,
+    then R_bd's off-block energy of H' (harp_off_block_energy, q = 128) and L_diag of the
+    rotated bf16 weight W' (28672 x 8192) weighted by diag(H') (harp_l_diag, qblock 128).
+    The two reductions read their matrix once: algorithmic bytes 4 n^2 and 2 n_out n_in."""
+    import numpy as np
+    n = w4.n_in
+    hdev = torch.from_numpy(W.draw_hessian(n, 4000 + w4.index).astype(np.float32)).to(device)
+    hrot = torch.empty_like(hdev)
+    ws = torch.empty(H.workspace_bytes(n, n), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    rot_ms = timed(lambda: H.apply_two_sided(pv, pv, hdev, hrot, ws))
+    e = torch.empty(2, dtype=torch.float64, device=device)
+    rbd_ms = timed(lambda: H.off_block_energy(hrot, q, e))
+    ld = torch.empty(1, dtype=torch.float64, device=device)
+    ldiag_ms = timed(lambda: H.l_diag(w_rot, hrot, q, ld))
+    ev = e.cpu().numpy()
+    b_rbd, b_ld = 4 * n * n, 2 * w_rot.numel()
+    del hdev, hrot, ws
+    return {"workload": f"fit terms on the two-sided shapes: H' = T_V^T H T_V ({n}x{n} fp32 Hessian proxy), "
+                        f"R_bd at q={q}, L_diag of W' ({w4.n_out}x{n} bf16) at qblock {q}",
+            "rotate_hessian_ms": rot_ms, "r_bd": float(ev[0] / ev[1]), "l_diag": float(ld.cpu().numpy()[0]),
+            "off_block_energy_ms": rbd_ms, "off_block_energy_hbm_gbs": b_rbd / (rbd_ms / 1e3) / 1e9,
+            "off_block_energy_hbm_frac": b_rbd / (rbd_ms / 1e3) / 1e9 / peak,
+            "l_diag_ms": ldiag_ms, "l_diag_hbm_gbs": b_ld / (ldiag_ms / 1e3) / 1e9,
+            "l_diag_hbm_frac": b_ld / (ldiag_ms / 1e3) / 1e9 / peak,
+            "kernel": "off_block_energy_kernel, l_diag_kernel"}
 
 
 def compose_measurement(args, H, W, torch, device, peak):

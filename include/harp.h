@@ -78,7 +78,7 @@ typedef enum {
     HARP_ERR_INVALID_ARG = 1,     /* null pointer, bad size, bad stride, partial aliasing */
     HARP_ERR_SCHEDULE = 2,        /* prod b_t != d, radix outside [2, 16], too many stages */
     HARP_ERR_UNSUPPORTED = 3,     /* dtype / direction value not known */
-    HARP_ERR_NOT_MATERIALIZED = 4,/* harp_apply before harp_materialize_blocks */
+    HARP_ERR_NOT_MATERIALIZED = 4,/* harp_apply before harp_materialize_blocks (float theta) */
     HARP_ERR_ALLOC = 5,           /* device or host allocation failed */
     HARP_ERR_CUDA = 6,            /* a CUDA runtime call or launch failed */
     HARP_ERR_TIMEOUT = 7,         /* a bounded device-side wait gave up */
@@ -118,7 +118,10 @@ HARP_API harp_status harp_plan_create(harp_plan_t* out, int64_t d, const int32_t
  * dequantized inside the kernel, §2.4).  Blocks are computed in double and stored
  * as float32; the sign diagonal is folded into the stage-0 blocks.  Allocates
  * device memory owned by the plan on first use.  Idempotent; a second call on
- * another device returns HARP_ERR_WRONG_DEVICE.
+ * another device returns HARP_ERR_WRONG_DEVICE.  Also builds, on `stream`, the
+ * coefficient table of the specialized d = 4096 (8,8,8,8) kernel for plans it covers,
+ * so that applies only read plan state.  Calls on one plan from several host threads
+ * take turns (a lock of the plan's).
  */
 HARP_API harp_status harp_materialize_blocks(harp_plan_t plan, void* stream);
 
@@ -134,10 +137,16 @@ HARP_API harp_status harp_materialize_blocks(harp_plan_t plan, void* stream);
  * multiply-adds (the specialized d = 4096 kernel forms the products on tensor cores from
  * TF32 hi/lo splits of both operands, three passes, fp32 accumulation), the output
  * rounded to `dtype` to nearest even.
- * Ordering: the first call that takes the specialized d = 4096 kernel for a plan (bf16,
- * FORWARD, 32 rows or more) builds that kernel's coefficient table on its stream; calls on
- * other streams must be ordered after that first call (an event or a synchronize), and
- * that first call must not run concurrently with another call on the same plan.
+ * Concurrency: a plan is immutable once materialized (every table a kernel reads is
+ * built by harp_materialize_blocks), so calls on different streams or host threads may
+ * run at once; order them after the materialization (same stream, an event or a
+ * synchronize).
+ * Materialization: a HARP_THETA_F32 plan that was not materialized returns
+ * HARP_ERR_NOT_MATERIALIZED.  A HARP_THETA_I8 plan materializes implicitly on its first
+ * call (its int8 codes are dequantized by the block-building kernel on the call's stream,
+ * which that call then synchronizes; concurrent first calls take turns on a lock of the
+ * plan and only one builds).  The same holds for every entry point below that takes a
+ * plan.
  */
 HARP_API harp_status harp_apply(harp_plan_t plan, const void* x, void* y, int64_t rows,
                        int64_t ld_x, int64_t ld_y, harp_dtype dtype, harp_dir dir,
@@ -245,8 +254,13 @@ HARP_API harp_status harp_apply_two_sided(harp_plan_t planU, harp_plan_t planV, 
  *   Limit: n_out * n_in <= HARP_NOALLOC_SCRATCH_BYTES / 8 elements (4,194,304),
  *          else HARP_ERR_INVALID_ARG and nothing is launched.
  *   First call on a device: looks up the array's device address
- *          (cudaGetSymbolAddress) with that device current; make that first call
- *          before any stream capture.
+ *          (cudaGetSymbolAddress) with that device current and keeps it for the
+ *          life of the process; make that first call before any stream capture.  The
+ *          kept address does not survive cudaDeviceReset: do not call this entry point
+ *          again after resetting the device in the same process.
+ *   Sides: each row pass holds one fp32 row in shared memory, so max(n_out, n_in) * 4
+ *          bytes must fit the device's opt-in shared memory per block (227 KiB on
+ *          B200), else HARP_ERR_UNSUPPORTED before anything is launched.
  *   Sharing: all calls use the same array; calls whose work overlaps on the GPU
  *          (different streams or host threads) race on it and must be serialized
  *          by the caller.  No part of the array needs to start at zero.
@@ -294,6 +308,46 @@ HARP_API harp_status harp_grad_theta(harp_plan_t plan, const void* x, const void
                                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * harp_off_block_energy — the block-diagonality term of the fit (§2.3 Optimization
+ * Objective: R_bd(Theta_V), the Hessian energy that falls outside the quantizer's blocks
+ * after the input-side rotation).  For a square matrix h of n x n (normally the rotated
+ * Hessian proxy H' = T_V^T H T_V, which is harp_apply_two_sided(planV, planV, H)):
+ *   out[0] = sum of h_ij^2 over i / q != j / q     (outside the q x q diagonal blocks)
+ *   out[1] = sum of all h_ij^2
+ * so R_bd = out[0] / out[1].  Squares and sums in double (fp32 and bf16 squares are exact
+ * there); the CTAs' partial sums are added with double atomics, so the last bits vary
+ * between runs.
+ *   h        device matrix, element type dtype, leading dimension ld >= n.
+ *   q        block size, q > 0 dividing n.
+ *   out      device array of 2 doubles, overwritten (zeroed on `stream` first); must not
+ *            overlap h.
+ * Asynchronous on `stream`; HARP_ERR_INVALID_ARG for bad sizes or NULL pointers.
+ */
+HARP_API harp_status harp_off_block_energy(const void* h, int64_t n, int64_t ld, harp_dtype dtype, int32_t q,
+                                           double* out, void* stream);
+
+/*
+ * harp_l_diag — the diagonal-weighted quantization error of the fit (§2.3 Optimization
+ * Objective: L_diag, the quantizer's error on the rotated weight weighted by the rotated
+ * Hessian's diagonal):
+ *   out[0] = sum_j h_jj sum_r (w_rj - Q(w)_rj)^2
+ * with Q the blockwise round-to-nearest int8 quantizer along the rows of w (per aligned
+ * block of qblock columns: s = max|w| / 127, code = clamp(round_half_even(w / s), -127,
+ * 127), Q(w) = code * s; a zero block is exact).  The quantizer's arithmetic is double
+ * (the same operations as its float64 definition, so its codes match that definition's
+ * for the same w); the sums are double with atomic adds across CTAs.
+ *   w        device rotated weight W' = T_U^T W T_V (harp_apply_two_sided), rows x cols,
+ *            element type dtype, leading dimension ld_w >= cols.
+ *   h        device float rotated Hessian proxy H' (cols x cols, leading dimension ld_h >=
+ *            cols); only its diagonal is read.
+ *   qblock   32, 64, 128 or 256, dividing cols.
+ *   out      device double, overwritten (zeroed on `stream` first); must not overlap w or h.
+ * rows = 0 writes 0.  Asynchronous on `stream`.
+ */
+HARP_API harp_status harp_l_diag(const void* w, int64_t rows, int64_t cols, int64_t ld_w, harp_dtype dtype,
+                                 const float* h, int64_t ld_h, int32_t qblock, double* out, void* stream);
+
+/*
  * harp_plan_compose — one plan for the composition T = T_{k-1} ... T_1 T_0 of k plans of
  * the same dimension (plans[0] acts first): k independent rotations in one pass over the
  * rows (composing two or three randomized Hadamard transforms brings every input's
@@ -330,6 +384,19 @@ HARP_API const char* harp_last_kernel(void);
 /* harp_last_error — detail of the last failing call on this host thread (static
  * per-thread buffer, valid until the next call). */
 HARP_API const char* harp_last_error(void);
+
+/*
+ * harp_test_inject_wait_timeout — test hook for the bounded device waits (the paper has no
+ * counterpart).  Until it is called again with (0, 0), every general tiled-kernel launch
+ * from this host thread tells its row-staging barriers to expect `extra_bytes` more than it
+ * copies and polls them only `poll_limit` times, so the first wait of each staged tile runs
+ * out: the kernel then sets the plan's status word (harp_plan_device_status reports
+ * HARP_ERR_TIMEOUT), retires the extra bytes itself, waits (bounded as usual) for the copies
+ * it really issued, and finishes with correct output.  No copy is left in flight and no
+ * wait is unbounded.  poll_limit >= 1 and 1 <= extra_bytes <= 4096, or both 0 to clear;
+ * else HARP_ERR_INVALID_ARG.
+ */
+HARP_API harp_status harp_test_inject_wait_timeout(int64_t poll_limit, uint32_t extra_bytes);
 
 /* ------------------------------------------------------------------------- */
 /* Host-side introspection: no device work, usable without a GPU.            */

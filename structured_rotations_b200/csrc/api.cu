@@ -95,8 +95,9 @@ harp_status apply_checked(harp_plan_t p, const void* x, void* y, int64_t rows, i
     if (ld_x < d || ld_y < d) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than d");
     if (rows == 0) return HARP_OK;
     if (!x || !y) return harp_fail(HARP_ERR_INVALID_ARG, "x or y is NULL");
-    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
-    harp_status st = check_device(p);
+    harp_status st = harp_require_materialized(p, stream);
+    if (st != HARP_OK) return st;
+    st = check_device(p);
     if (st != HARP_OK) return st;
     const size_t es_in = esize(in_dtype), es_out = esize(out_dtype);
     if (x == y) {
@@ -138,8 +139,9 @@ extern "C" harp_status harp_apply_quant(harp_plan_t p, const void* x, int64_t ro
         return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than the row");
     if (rows == 0) return HARP_OK;
     if (!x || !q || !scales) return harp_fail(HARP_ERR_INVALID_ARG, "x, q or scales is NULL");
-    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
-    harp_status st = check_device(p);
+    harp_status st = harp_require_materialized(p, stream);
+    if (st != HARP_OK) return st;
+    st = check_device(p);
     if (st != HARP_OK) return st;
     const size_t xb = ((rows - 1) * ld_x + d) * 2, qb = (rows - 1) * ld_q + d,
                  sb = ((rows - 1) * ld_s + d / qblock) * sizeof(float);
@@ -163,8 +165,9 @@ extern "C" harp_status harp_apply_columns(harp_plan_t p, float* x, int64_t ld_x,
     if (ld_x < ncols || ld_y < ncols) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than ncols");
     if (ncols == 0) return HARP_OK;
     if (!x || !y) return harp_fail(HARP_ERR_INVALID_ARG, "x or y is NULL");
-    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
-    harp_status st = check_device(p);
+    harp_status st = harp_require_materialized(p, stream);
+    if (st != HARP_OK) return st;
+    st = check_device(p);
     if (st != HARP_OK) return st;
     const int64_t d = p->desc.d;
     const size_t xb = ((d - 1) * ld_x + ncols) * sizeof(float), yb = ((d - 1) * ld_y + ncols) * esize(out_dtype);
@@ -200,9 +203,9 @@ extern "C" harp_status harp_apply_two_sided(harp_plan_t pu, harp_plan_t pv, cons
     if (((uintptr_t)workspace & 255) != 0) return harp_fail(HARP_ERR_INVALID_ARG, "workspace not 256-byte aligned");
     if (ws_bytes < harp_two_sided_workspace_bytes(n_out, n_in))
         return harp_fail(HARP_ERR_INVALID_ARG, "workspace too small");
-    if (!pu->materialized || !pv->materialized)
-        return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks on both plans");
     harp_status st;
+    if ((st = harp_require_materialized(pu, stream)) != HARP_OK || (st = harp_require_materialized(pv, stream)) != HARP_OK)
+        return st;
     if ((st = check_device(pu)) != HARP_OK || (st = check_device(pv)) != HARP_OK) return st;
     const size_t es = esize(dtype);
     const size_t wbytes = ((n_out - 1) * ld + n_in) * es;

@@ -610,13 +610,10 @@ bool is_d4096_radix8(const harp_plan_s* p) {
     return true;
 }
 
+// The coefficient table and the launch attributes of the specialized kernel, built once per
+// plan by materialization (on the materializing stream): afterwards launches only read
+// them, so calls on any number of streams may run at once.
 harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
-    FastState* fs = static_cast<FastState*>(p->fast);
-    if (fs && fs->ready) return HARP_OK;
-    if (!fs) {
-        fs = new FastState();
-        p->fast = fs;
-    }
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult qres;
@@ -626,18 +623,12 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
         cudaGetLastError();
     });
     if (!g_encode) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-    const int nfloat = 2 * kWarps * 128 * 32;
-    if (!fs->frag && cudaMalloc((void**)&fs->frag, sizeof(float) * nfloat) != cudaSuccess) {
-        cudaGetLastError();
-        return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the fragment table failed");
-    }
-    const float* blocks = p->d_blocks;
-    pack_fragments_kernel<<<(nfloat + 255) / 256, 256, 0, stream>>>(
-        blocks + p->desc.st[0].block_off, blocks + p->desc.st[1].block_off, blocks + p->desc.st[2].block_off,
-        blocks + p->desc.st[3].block_off, fs->frag);
     cudaError_t e = cudaFuncSetAttribute(harp_fast_d4096_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
-    if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2);
     cfg.blockDim = dim3(kThreads);
@@ -648,10 +639,26 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
         cudaGetLastError();
         return harp_fail(HARP_ERR_CUDA, "no cluster of two fits on this device");
     }
-    fs->max_pairs = nclusters;
+    FastState* fs = new FastState();
+    const int nfloat = 2 * kWarps * 128 * 32;
+    if (cudaMalloc((void**)&fs->frag, sizeof(float) * nfloat) != cudaSuccess) {
+        cudaGetLastError();
+        delete fs;
+        return harp_fail(HARP_ERR_ALLOC, "cudaMalloc of the fragment table failed");
+    }
+    const float* blocks = p->d_blocks;
+    pack_fragments_kernel<<<(nfloat + 255) / 256, 256, 0, stream>>>(
+        blocks + p->desc.st[0].block_off, blocks + p->desc.st[1].block_off, blocks + p->desc.st[2].block_off,
+        blocks + p->desc.st[3].block_off, fs->frag);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    if (e != cudaSuccess) {
+        cudaFree(fs->frag);
+        delete fs;
+        return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    }
+    fs->max_pairs = nclusters;
     fs->ready = true;
+    p->fast = fs;
     return HARP_OK;
 }
 
@@ -666,9 +673,8 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     if (((uintptr_t)x & 15) || (ld_x & 7) || ((uintptr_t)y & 15) || (ld_y & 7)) return HARP_ERR_UNSUPPORTED;
     if (rows < 32 || rows > 0x7fffffffll) return HARP_ERR_UNSUPPORTED;
     cudaStream_t stream = (cudaStream_t)stream_;
-    harp_status st = prepare(p, stream);
-    if (st != HARP_OK) return st;
-    FastState* fs = static_cast<FastState*>(p->fast);
+    const FastState* fs = static_cast<const FastState*>(p->fast);
+    if (!fs || !fs->ready) return HARP_ERR_UNSUPPORTED;   // no table: the plan was not eligible or it failed
     const int64_t ntiles = (rows + kTile - 1) / kTile;
     const int pairs = (int)std::min<int64_t>(fs->max_pairs, ntiles);
 
@@ -677,9 +683,18 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     const cuuint64_t gstride[1] = {(cuuint64_t)ld_x * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
     const cuuint32_t estride[2] = {1, 1};
-    CUresult cr = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box,
-                           estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    auto encode = [&] {
+        return g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    };
+    CUresult cr = encode();
+    if (cr == CUDA_ERROR_INVALID_CONTEXT) {
+        // a host thread whose first CUDA call this is has no current context yet: bind the
+        // plan's device (the runtime's primary context) and encode again
+        if (cudaSetDevice(p->device) != cudaSuccess) cudaGetLastError();
+        cr = encode();
+    }
     if (cr != CUDA_SUCCESS) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)cr));
 
     FastParams fp;
@@ -694,6 +709,11 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_fast_d4096_fwd_kernel");
     return HARP_OK;
+}
+
+void fast_prepare(harp_plan_s* p, void* stream) {
+    if (p->fast || !is_d4096_radix8(p)) return;
+    if (prepare(p, (cudaStream_t)stream) != HARP_OK) harp_clear_error();   // the plan runs on the tiled kernel
 }
 
 void fast_state_free(harp_plan_s* p) {

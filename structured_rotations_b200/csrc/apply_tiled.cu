@@ -53,7 +53,23 @@ int sm_count() {
     return cached[dev];
 }
 
+// Test hook (harp_test_inject_wait_timeout): the poll limit and over-declared bytes of the
+// next tiled launches on this host thread.
+thread_local long long g_inject_limit = 0;
+thread_local uint32_t g_inject_extra = 0;
+
 }  // namespace
+
+extern "C" harp_status harp_test_inject_wait_timeout(int64_t poll_limit, uint32_t extra_bytes) {
+    harp_clear_error();
+    // the barrier's transaction count holds less than 2^20 bytes: the staged rows (under
+    // 227 KiB) plus at most 4 KiB stay below it
+    if (poll_limit < 0 || (extra_bytes != 0 && poll_limit == 0) || extra_bytes > 4096)
+        return harp_fail(HARP_ERR_INVALID_ARG, "poll_limit >= 1 with 1..4096 extra bytes, or (0, 0) to clear");
+    g_inject_limit = extra_bytes ? poll_limit : 0;
+    g_inject_extra = extra_bytes;
+    return HARP_OK;
+}
 
 harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
                                int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
@@ -156,6 +172,8 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.staged_rows = (int)staged;
     tp.mask = (dl % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
+    tp.wait_limit = g_inject_extra ? g_inject_limit : kWaitLimit;
+    tp.extra_tx = g_inject_extra;
     tp.last_blocks = p->d_blocks + pd.st[pd.m - 1].block_off;
     for (int t = 0; t < pd.m; ++t) {
         tp.nb_div[t] = make_fast_div((int)(dl / pd.st[t].b));

@@ -71,6 +71,9 @@ struct TiledParams {
     float* scales;                     // quantized output (int8 codes in y): per-block scales
     int64_t ld_s;                      // scales per row of the scales array (row stride)
     int qlanes;                        // quantizer block / 8: lanes that hold one block
+    long long wait_limit;              // polls of a staging wait before it gives up (kWaitLimit)
+    uint32_t extra_tx;                 // test hook, normally 0: bytes each staging barrier is told to
+                                       // expect beyond what is copied, so its first wait runs out
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -89,10 +92,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-// Bounded wait for the phase with the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Retires `bytes` of a barrier's expected transaction count without a copy.
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bounded wait for the phase with the given parity; false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kWaitLimit) {
     const uint32_t addr = smem_u32(bar);
-    for (long long i = 0; i < kWaitLimit; ++i) {
+    for (long long i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
             "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
@@ -323,7 +332,7 @@ __device__ __forceinline__ void issue_tile(const TiledParams& p, int64_t tile, i
     const int64_t row0 = tile * p.R;
     const int nr = (int)min((int64_t)p.staged_rows, p.rows - row0);
     const uint32_t row_bytes = (uint32_t)dl * sizeof(TIn);
-    mbar_arrive_expect_tx(bar, row_bytes * nr);
+    mbar_arrive_expect_tx(bar, row_bytes * nr + p.extra_tx);
     const TIn* x = (const TIn*)p.x + col0;
     for (int r = 0; r < nr; ++r) bulk_load(stage_buf + (size_t)r * row_bytes, x + (row0 + r) * p.ld_x, row_bytes, bar);
 }
@@ -575,12 +584,20 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         const int qv = (nr + V - 1) / V;
         const int n_staged = min(nr, p.staged_rows);
         if (n_staged && !failed) {
-            const bool ok = mbar_wait(bar, parity);
-            parity ^= 1;
+            bool ok = mbar_wait(bar, parity, p.wait_limit);
             if (__syncthreads_or(!ok)) {
                 if (tid == 0) atomicExch(p.status, 1);
-                failed = true;
+                if (p.extra_tx) {
+                    // the test hook's over-declared bytes: retire them, then wait (bounded)
+                    // for the copies that were really issued, and go on with correct data
+                    if (tid == 0) mbar_complete_tx(bar, p.extra_tx);
+                    ok = mbar_wait(bar, parity, kWaitLimit);
+                    failed = __syncthreads_or(!ok);
+                } else {
+                    failed = true;
+                }
             }
+            parity ^= 1;
         }
         fill_tile<V, NT, TIn>(tile, dl, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x + col0,
                               p.ld_x, p.mask);

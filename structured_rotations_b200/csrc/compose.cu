@@ -27,9 +27,10 @@ extern "C" harp_status harp_plan_compose(harp_plan_t* out, const harp_plan_t* pl
     int64_t d = -1;
     int m = 0;
     for (int j = 0; j < k; ++j) {
-        const harp_plan_s* p = plans[j];
+        harp_plan_s* p = plans[j];
         if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "a plan is NULL");
-        if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "materialize every plan first");
+        const harp_status mst = harp_require_materialized(plans[j], stream_);   // int8 plans: implicitly
+        if (mst != HARP_OK) return mst;
         if (p->device != dev) return harp_fail(HARP_ERR_WRONG_DEVICE, "plans must be materialized on the current device");
         if (d >= 0 && p->desc.d != d) return harp_fail(HARP_ERR_INVALID_ARG, "plans of different dimensions");
         d = p->desc.d;
@@ -84,6 +85,10 @@ extern "C" harp_status harp_plan_compose(harp_plan_t* out, const harp_plan_t* pl
                                 cudaMemcpyDeviceToDevice, stream);
         boff += p->block_floats;
         loff += p->lane_floats;
+    }
+    if (e == cudaSuccess) {
+        fast_prepare(c, stream);   // a composite of one (8,8,8,8) plan of d = 4096 takes the specialized kernel
+        e = cudaGetLastError();
     }
     // wait for the copies, so that the source plans may be destroyed as soon as this returns
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);

@@ -410,7 +410,10 @@ extern "C" harp_status harp_grad_theta(harp_plan_t p, const void* x, const void*
     if (ld_x < d || ld_g < d) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than d");
     if (!dtheta) return harp_fail(HARP_ERR_INVALID_ARG, "dtheta is NULL");
     if (p->composite) return harp_fail(HARP_ERR_UNSUPPORTED, "the gradient is taken for one plan, not a composite");
-    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    {
+        const harp_status mst = harp_require_materialized(p, stream);
+        if (mst != HARP_OK) return mst;
+    }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -424,6 +427,19 @@ extern "C" harp_status harp_grad_theta(harp_plan_t p, const void* x, const void*
         return harp_fail(HARP_ERR_INVALID_ARG, "workspace smaller than harp_grad_workspace_bytes()");
     if (((uintptr_t)workspace & 15) != 0) return harp_fail(HARP_ERR_INVALID_ARG, "workspace not 16-byte aligned");
     if (rows > 0 && (!x || !g)) return harp_fail(HARP_ERR_INVALID_ARG, "x or g is NULL");
+    {
+        // the accumulators are zeroed and then added to while x and g are read, and dtheta is
+        // written last: none of them may share memory with another
+        const size_t es = dtype == HARP_F32 ? 4 : 2;
+        const size_t xb = rows > 0 ? ((size_t)(rows - 1) * ld_x + d) * es : 0;
+        const size_t gb = rows > 0 ? ((size_t)(rows - 1) * ld_g + d) * es : 0;
+        const size_t tb = (size_t)p->theta_total * sizeof(float);
+        if (rows > 0 && (ranges_overlap(workspace, ws_bytes, x, xb) || ranges_overlap(workspace, ws_bytes, g, gb)))
+            return harp_fail(HARP_ERR_INVALID_ARG, "workspace overlaps x or g");
+        if (ranges_overlap(dtheta, tb, workspace, ws_bytes) ||
+            (rows > 0 && (ranges_overlap(dtheta, tb, x, xb) || ranges_overlap(dtheta, tb, g, gb))))
+            return harp_fail(HARP_ERR_INVALID_ARG, "dtheta overlaps the workspace, x or g");
+    }
     // rows per tile: two fp32 tiles of rows rounded up to 32 coordinates (the swizzle
     // permutes aligned blocks of 32) within the 227 KiB of shared memory a CTA may use
     const int rs = (int)((d + 31) / 32 * 32);

@@ -1,6 +1,7 @@
 // Internal declarations shared by the host plan code and the CUDA launchers.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <map>
 #include <mutex>
@@ -47,7 +48,10 @@ struct harp_plan_s {
 
     // device side (owned)
     int device = -1;
-    bool materialized = false;
+    // Set last by materialization, once the blocks (and every table a kernel reads) are
+    // built; atomic so that a call that sees it set also sees the finished device state.
+    std::atomic<bool> materialized{false};
+    std::mutex materialize_mu;        // explicit and implicit (int8) materialization take turns
     bool composite = false;           // built by harp_plan_compose: stages of several plans in a row
     float* d_blocks = nullptr;        // signed blocks, [stage][c][k][l]
     float* d_blocks_lanes = nullptr;  // the same, lane-interleaved (see lane_off)
@@ -61,6 +65,9 @@ struct harp_plan_s {
     std::mutex host_io_mu;            // harp_apply_host calls on this plan take turns
 };
 
+// true if the byte ranges [a, a + na) and [b, b + nb) share a byte (api.cu)
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb);
+
 // error reporting (plan.cpp)
 harp_status harp_fail(harp_status s, const std::string& msg);
 void harp_clear_error();
@@ -72,6 +79,11 @@ int harp_set_smem_limit(const void* kernel, int bytes);
 
 // device helpers (materialize.cu)
 harp_status harp_device_free(harp_plan_s* p);
+// HARP_OK if the plan is materialized.  An int8 plan that is not is materialized here on
+// `stream`, which is then synchronized before the plan is marked ready, so that a call
+// from another stream or thread that finds it ready reads finished blocks.  Other plans
+// return HARP_ERR_NOT_MATERIALIZED.
+harp_status harp_require_materialized(harp_plan_s* p, void* stream);
 
 // launchers (apply_simple.cu / transpose.cu)
 harp_status launch_apply_simple(const harp_plan_s* p, const void* x, void* y, int64_t rows,
@@ -87,6 +99,11 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               int64_t ld_x, int64_t ld_y, harp_dtype in_dtype, harp_dir dir,
                               void* stream, harp_dtype out_dtype);
 void fast_state_free(harp_plan_s* p);
+// Builds the specialized kernel's coefficient table (and its launch attributes) on
+// `stream` for plans it covers; a no-op for other plans.  Called by materialization, so
+// every later launch only reads the table.  A plan whose table cannot be built (no
+// cluster fits, no tensor-map encoder) is left without one and runs on the other kernels.
+void fast_prepare(harp_plan_s* p, void* stream);
 void host_io_free(harp_plan_s* p);
 
 // the row kernels in order of preference (api.cu)

@@ -5,6 +5,7 @@
 // so the two copy directions (separate copy engines) and the kernels run at once.
 #include <algorithm>
 #include <mutex>
+#include <string>
 
 #include <cuda_runtime.h>
 
@@ -88,7 +89,11 @@ extern "C" harp_status harp_apply_host(harp_plan_t p, const void* x, void* y, in
     if (ld_x < d || ld_y < d) return harp_fail(HARP_ERR_INVALID_ARG, "leading dimension smaller than d");
     if (rows == 0) return HARP_OK;
     if (!x || !y) return harp_fail(HARP_ERR_INVALID_ARG, "x or y is NULL");
-    if (!p->materialized) return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    {
+        // int8 plans materialize on their first call (on the legacy stream, synchronized)
+        const harp_status mst = harp_require_materialized(p, nullptr);
+        if (mst != HARP_OK) return mst;
+    }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -110,6 +115,14 @@ extern "C" harp_status harp_apply_host(harp_plan_t p, const void* x, void* y, in
     harp_status st = ensure(p, (size_t)chunk * row_bytes);
     if (st != HARP_OK) return st;
     HostIo* h = (HostIo*)p->host_io;
+    // On an error after the first enqueue, the earlier chunks' copies may still be reading x
+    // or writing y: wait for all three streams before returning, so the caller may free or
+    // reuse its buffers at once.
+    auto drain_and_fail = [&](harp_status s, const std::string& msg) {
+        for (int i = 0; i < kSlots; ++i) cudaStreamSynchronize(h->stream[i]);
+        cudaGetLastError();
+        return harp_fail(s, msg);
+    };
     const char* xs = (const char*)x;
     char* ys = (char*)y;
     int64_t k = 0;
@@ -119,22 +132,18 @@ extern "C" harp_status harp_apply_host(harp_plan_t p, const void* x, void* y, in
         const int64_t n = std::min(chunk, rows - r0);
         cudaError_t e = cudaMemcpy2DAsync(h->din[slot], row_bytes, xs + (size_t)r0 * ld_x * es, (size_t)ld_x * es,
                                           row_bytes, (size_t)n, cudaMemcpyHostToDevice, s);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
-        }
+        if (e != cudaSuccess) return drain_and_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
         st = run_rows(p, h->din[slot], h->dout[slot], n, d, d, dtype, dtype, dir, s);
-        if (st != HARP_OK) return st;
+        if (st != HARP_OK) return drain_and_fail(st, harp_last_error());
         e = cudaMemcpy2DAsync(ys + (size_t)r0 * ld_y * es, (size_t)ld_y * es, h->dout[slot], row_bytes, row_bytes,
                               (size_t)n, cudaMemcpyDeviceToHost, s);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
-        }
+        if (e != cudaSuccess) return drain_and_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     }
+    cudaError_t first = cudaSuccess;
     for (int i = 0; i < kSlots; ++i) {
         const cudaError_t e = cudaStreamSynchronize(h->stream[i]);
-        if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+        if (e != cudaSuccess && first == cudaSuccess) first = e;
     }
+    if (first != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(first));
     return HARP_OK;
 }

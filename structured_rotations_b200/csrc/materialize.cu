@@ -5,6 +5,8 @@
 //   B = Q G_b, with stage 0's columns multiplied by the sign diagonal S,
 // in double, and stores B as float32.  int8 parameters are dequantized here
 // (q * scale_t), so theta stays in its storage form until this kernel.
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 #include "harp_internal.h"
@@ -137,9 +139,11 @@ harp_status harp_device_free(harp_plan_s* p) {
     return cudaGetLastError() == cudaSuccess ? HARP_OK : HARP_ERR_CUDA;
 }
 
-extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream_) {
-    harp_clear_error();
-    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+namespace {
+
+// Uploads and builds everything on `stream_`; the caller holds the plan's materialize_mu
+// and sets p->materialized afterwards.
+harp_status materialize_locked(harp_plan_s* p, void* stream_) {
     cudaStream_t stream = (cudaStream_t)stream_;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -199,9 +203,38 @@ extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream_) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    fast_prepare(p, stream);   // the specialized kernel's table, so that launches only read plan state
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    return HARP_OK;
+}
+
+}  // namespace
+
+extern "C" harp_status harp_materialize_blocks(harp_plan_t p, void* stream) {
+    harp_clear_error();
+    if (!p) return harp_fail(HARP_ERR_INVALID_ARG, "plan is NULL");
+    std::lock_guard<std::mutex> lock(p->materialize_mu);
+    const harp_status st = materialize_locked(p, stream);
+    if (st == HARP_OK) p->materialized = true;
+    return st;
+}
+
+harp_status harp_require_materialized(harp_plan_s* p, void* stream) {
+    if (p->materialized) return HARP_OK;
+    if (p->kind != HARP_THETA_I8)
+        return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks first");
+    std::lock_guard<std::mutex> lock(p->materialize_mu);
+    if (p->materialized) return HARP_OK;   // another call got there first (and synchronized)
+    harp_status st = materialize_locked(p, stream);
+    if (st != HARP_OK) return st;
+    const cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     p->materialized = true;
     return HARP_OK;
 }
+
+
 
 extern "C" harp_status harp_plan_device_status(harp_plan_t p) {
     harp_clear_error();

@@ -12,7 +12,9 @@
 // calls whose work overlaps on the GPU (two streams, or two host threads) race on
 // it, so serialize them.  Nothing in it has to start at zero: every byte a call
 // reads was written earlier by the same call.
+#include <algorithm>
 #include <mutex>
+#include <string>
 
 #include <cuda_runtime.h>
 
@@ -30,7 +32,9 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // symbol is only a host-side stand-in, so the address is looked up once per device
-// with that device current.
+// with that device current and kept for the life of the process; it does not survive
+// cudaDeviceReset (the module may come back at another address), after which this
+// entry point must not be called again in the same process.
 harp_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -78,8 +82,9 @@ extern "C" harp_status harp_apply_two_sided_noalloc(harp_plan_t pu, harp_plan_t 
         return harp_fail(HARP_ERR_INVALID_ARG,
                          "weight too large for the static scratch: n_out * n_in must be at most " +
                              std::to_string(kScratchBytes / 8) + " elements");
-    if (!pu->materialized || !pv->materialized)
-        return harp_fail(HARP_ERR_NOT_MATERIALIZED, "call harp_materialize_blocks on both plans");
+    harp_status st;
+    if ((st = harp_require_materialized(pu, stream)) != HARP_OK || (st = harp_require_materialized(pv, stream)) != HARP_OK)
+        return st;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -92,8 +97,20 @@ extern "C" harp_status harp_apply_two_sided_noalloc(harp_plan_t pu, harp_plan_t 
     if (W != W_out && overlap(W, wbytes, W_out, wbytes))
         return harp_fail(HARP_ERR_INVALID_ARG, "W and W_out overlap without being equal");
 
+    {
+        // each row pass holds one whole fp32 row in shared memory: check the longer side against
+        // the device's opt-in limit now, before anything is enqueued
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return harp_fail(HARP_ERR_CUDA, "cannot read the shared-memory limit");
+        }
+        if ((size_t)std::max(n_out, n_in) * sizeof(float) > (size_t)optin)
+            return harp_fail(HARP_ERR_UNSUPPORTED, "a side of the weight is too long for one fp32 row in shared memory (" +
+                                                       std::to_string(optin / 4) + " elements at most)");
+    }
     void* scratch = nullptr;
-    harp_status st = scratch_address(&scratch);
+    st = scratch_address(&scratch);
     if (st != HARP_OK) return st;
     float* ws1 = (float*)scratch;
     float* ws2 = (float*)((char*)scratch + half);

@@ -79,6 +79,9 @@ def lib():
                                       _vp]),
         "harp_grad_theta": (_c_i32, [_vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _vp, ctypes.c_size_t,
                                      _vp]),
+        "harp_off_block_energy": (_c_i32, [_vp, _c_i64, _c_i64, _c_i32, _c_i32, _vp, _vp]),
+        "harp_l_diag": (_c_i32, [_vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _c_i64, _c_i32, _vp, _vp]),
+        "harp_test_inject_wait_timeout": (_c_i32, [_c_i64, ctypes.c_uint32]),
         "harp_plan_destroy": (_c_i32, [_vp]),
         "harp_status_string": (ctypes.c_char_p, [_c_i32]),
         "harp_last_error": (ctypes.c_char_p, []),
@@ -374,3 +377,37 @@ def apply_two_sided(plan_u: Plan, plan_v: Plan, w, w_out=None, workspace=None, s
                                       workspace.numel() * workspace.element_size(),
                                       _stream_handle(stream)), "harp_apply_two_sided")
     return w_out
+
+
+def off_block_energy(h, q: int, out=None, stream=None):
+    """(energy of the square matrix h outside its q x q diagonal blocks, total energy) as a
+    device float64 tensor of 2 (harp_off_block_energy); R_bd = out[0] / out[1]."""
+    import torch
+    n = h.shape[0]
+    if h.dim() != 2 or h.shape[1] != n:
+        raise ValueError("h must be square")
+    if out is None:
+        out = torch.empty(2, dtype=torch.float64, device=h.device)
+    _check(lib().harp_off_block_energy(h.data_ptr(), n, _ld(h), _dtype_code(h), q, out.data_ptr(),
+                                       _stream_handle(stream)), "harp_off_block_energy")
+    return out
+
+
+def l_diag(w, h, qblock: int, out=None, stream=None):
+    """sum_j h_jj sum_r (w_rj - Q(w)_rj)^2 with Q the blockwise int8 quantizer along the rows
+    (harp_l_diag), as a device float64 tensor of 1; h is float32 (only its diagonal is read)."""
+    import torch
+    rows, cols = w.shape
+    if h.dtype != torch.float32 or h.shape[0] < cols or h.shape[1] < cols:
+        raise ValueError("h must be a float32 matrix of at least cols x cols")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float64, device=w.device)
+    _check(lib().harp_l_diag(w.data_ptr(), rows, cols, _ld(w), _dtype_code(w), h.data_ptr(), _ld(h), qblock,
+                             out.data_ptr(), _stream_handle(stream)), "harp_l_diag")
+    return out
+
+
+def inject_wait_timeout(poll_limit: int = 0, extra_bytes: int = 0) -> None:
+    """Test hook (harp_test_inject_wait_timeout): make the staging waits of this thread's
+    next tiled-kernel launches run out after poll_limit polls; (0, 0) clears it."""
+    _check(lib().harp_test_inject_wait_timeout(poll_limit, extra_bytes), "harp_test_inject_wait_timeout")

@@ -189,3 +189,31 @@ def test_plan_compose_argument_errors_before_any_device_call():
     assert L.harp_plan_compose(ctypes.byref(out), plans, 0, None) == HB.HARP_ERR_INVALID_ARG
     assert L.harp_plan_compose(ctypes.byref(out), None, 1, None) == HB.HARP_ERR_INVALID_ARG
     assert not out.value
+
+
+def test_wait_timeout_hook_arguments():
+    L = H.lib()
+    assert L.harp_test_inject_wait_timeout(0, 16) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_test_inject_wait_timeout(-1, 0) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_test_inject_wait_timeout(10, 8192) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_test_inject_wait_timeout(5, 16) == HB.HARP_OK
+    assert L.harp_test_inject_wait_timeout(0, 0) == HB.HARP_OK
+
+
+def test_fit_term_argument_errors_before_any_device_call():
+    L = H.lib()
+    p = ctypes.c_void_p(16)
+    out = ctypes.c_void_p(1 << 40)
+    assert L.harp_off_block_energy(p, 64, 64, HB.HARP_F32, 48, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_off_block_energy(p, 64, 63, HB.HARP_F32, 8, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_off_block_energy(p, 0, 64, HB.HARP_F32, 8, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_off_block_energy(p, 64, 64, 9, 8, out, None) == HB.HARP_ERR_UNSUPPORTED
+    assert L.harp_off_block_energy(None, 64, 64, HB.HARP_F32, 8, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_off_block_energy(p, 64, 64, HB.HARP_F32, 8, ctypes.c_void_p(32), None) == HB.HARP_ERR_INVALID_ARG
+    for qb in (16, 48, 512):
+        assert L.harp_l_diag(p, 4, 512, 512, HB.HARP_F32, p, 512, qb, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_l_diag(p, 4, 96, 96, HB.HARP_F32, p, 96, 64, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_l_diag(p, 4, 512, 511, HB.HARP_F32, p, 512, 32, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_l_diag(p, 4, 512, 512, HB.HARP_F32, p, 511, 32, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_l_diag(p, 4, 512, 512, HB.HARP_F32, None, 512, 32, out, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_l_diag(p, 4, 512, 512, 3, p, 512, 32, out, None) == HB.HARP_ERR_UNSUPPORTED

@@ -5,8 +5,9 @@ Some callers cannot allocate device memory at the moment they rotate a weight
 runtimes without an allocator for plugins), so the library offers a variant of
 the two-sided rotation whose workspace is a fixed array in its own device image.
 These tests call it through the C ABI and hold its output to the same tolerance
-as every other bf16 test, against the workspace-taking entry point, on two calls
-in a row.  The file is named to be collected last.
+as every other bf16 test: within one bf16 ordinal step of the float64 oracle's
+T_U^T W T_V (tests/_parity.check_bf16), and within one step of the workspace-taking
+entry point, on two calls in a row.  The file is named to be collected last.
 """
 import ctypes
 
@@ -15,10 +16,11 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
+from oracle import harp_oracle as O
 import workloads as W
 import structured_rotations_b200 as H
 from structured_rotations_b200 import harp as HB
-from tests._parity import bf16_ordinal
+from tests._parity import bf16_ordinal, check_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -27,6 +29,11 @@ def _plan(sched, seed, sign):
     d = int(np.prod(sched))
     theta = W.draw_theta(H.theta_count(sched), 0.2236, seed)
     return H.Plan(d, sched, theta=theta, sign_seed=sign).materialize()
+
+
+def _oracle_plan(sched, seed, sign):
+    d = int(np.prod(sched))
+    return O.make_plan(d, sched, W.draw_theta(O.theta_count(sched), 0.2236, seed), sign_seed=sign)
 
 
 def _as_bits(t):
@@ -40,9 +47,12 @@ def test_noalloc_matches_workspace_entry_point_twice(u_sched, v_sched):
     n_out, n_in = pu.d, pv.d
     assert n_out * n_in * 8 <= L.harp_noalloc_scratch_bytes()
     rng = np.random.default_rng(n_out + n_in)
-    w = torch.from_numpy(W.encode_bf16(0.02 * rng.standard_normal((n_out, n_in))).view(np.int16))
-    w = w.view(torch.bfloat16).cuda()
+    enc = W.encode_bf16(0.02 * rng.standard_normal((n_out, n_in)))
+    w = torch.from_numpy(enc.view(np.int16)).view(torch.bfloat16).cuda()
     ref = _as_bits(H.apply_two_sided(pu, pv, w))
+    wv = W.decode_bf16(enc)
+    exact = O.two_sided(_oracle_plan(u_sched, 41, 5), _oracle_plan(v_sched, 42, 6), wv)
+    wnorm = np.full(n_out, np.max(np.linalg.norm(wv, axis=1)))   # the two-sided tests' row-norm scale
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
         out = torch.empty_like(w)
@@ -51,6 +61,7 @@ def test_noalloc_matches_workspace_entry_point_twice(u_sched, v_sched):
         assert st == HB.HARP_OK, L.harp_last_error()
         torch.cuda.synchronize()
         got = _as_bits(out)
+        check_bf16(got, exact, wnorm, O.round_bf16, "noalloc against the oracle")
         assert np.abs(bf16_ordinal(got) - bf16_ordinal(ref)).max() <= 1
 
 

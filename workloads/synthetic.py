@@ -41,7 +41,7 @@ ROW_BLOCK = 256
 __all__ = [
     "ROW_BLOCK", "Workload", "WORKLOADS", "get", "draw_rows", "draw_theta",
     "encode_bf16", "decode_bf16", "quantize_theta_int8", "sample_rows",
-    "draw_weight", "draw_encoded", "draw_upstream", "C5_ROWS",
+    "draw_weight", "draw_encoded", "draw_upstream", "C5_ROWS", "draw_hessian",
 ]
 
 
@@ -281,6 +281,18 @@ def draw_upstream(w: Workload, row_start: int = 0, row_count: Optional[int] = No
 def draw_weight(w: Workload) -> np.ndarray:
     """The two-sided workload's weight matrix W (n_out x n_in), float64 values."""
     return draw_rows(w, 0, w.n_out, w.n_in)
+
+
+def draw_hessian(n: int, seed: int, samples: int = 256) -> np.ndarray:
+    """A seeded symmetric positive definite Hessian proxy of n x n (float64, values exact
+    in float32): X^T X / samples + 0.01 I for calibration-like activations X (samples x n,
+    iid N(0, 1) with 8 seeded outlier channels x20), rounded to float32 and symmetric."""
+    rng = np.random.default_rng([seed, 0x4E55])
+    x = rng.standard_normal((samples, n))
+    x[:, np.sort(rng.choice(n, size=min(8, n), replace=False))] *= 20.0
+    h = x.T @ x / samples + 0.01 * np.eye(n)
+    h = 0.5 * (h + h.T)
+    return h.astype(np.float32).astype(np.float64)
 
 
 def sample_rows(rows: int, count: int, seed: int = 7) -> np.ndarray:
