@@ -28,9 +28,10 @@ harp_status check_device(const harp_plan_s* p) {
 }
 
 // HARP_KERNEL selects the row kernel: unset = the fastest one that covers the shape
-// (specialized, then tiled, then simple); "simple", "tiled" or "fast" (specialized) force
-// one and fail with HARP_ERR_UNSUPPORTED if it does not cover the shape.
-enum { kAuto = 0, kSimple = 1, kFast = 2, kTiled = 3 };
+// (specialized, then the cluster kernel for small batches, then tiled, then simple);
+// "simple", "tiled", "cluster" or "fast" (specialized) force one and fail with
+// HARP_ERR_UNSUPPORTED if it does not cover the shape.
+enum { kAuto = 0, kSimple = 1, kFast = 2, kTiled = 3, kCluster = 4 };
 
 int kernel_choice() {
     const char* v = std::getenv("HARP_KERNEL");
@@ -38,8 +39,14 @@ int kernel_choice() {
     if (!std::strcmp(v, "simple")) return kSimple;
     if (!std::strcmp(v, "fast")) return kFast;
     if (!std::strcmp(v, "tiled")) return kTiled;
+    if (!std::strcmp(v, "cluster")) return kCluster;
     return kAuto;
 }
+
+// Batches below this many rows take the cluster kernel when the plan has one: their cost is
+// the blocks' reads, which the cluster spreads over its CTAs (measured on B200: 1 and 16 rows of
+// d = 4096 / 5120 / 8192 faster on it, 256 rows of d = 4096 and 8192 faster on the tiled kernel).
+constexpr int64_t kClusterRows = 65;
 
 }  // namespace
 
@@ -64,6 +71,11 @@ harp_status run_rows(harp_plan_s* p, const void* x, void* y, int64_t rows, int64
     if (choice == kAuto || choice == kFast) {
         st = launch_apply_fast(p, x, y, rows, ld_x, ld_y, in_dtype, dir, stream, out_dtype);
         if (st != HARP_ERR_UNSUPPORTED || choice == kFast) return st;
+        harp_clear_error();
+    }
+    if (choice == kCluster || (choice == kAuto && rows < kClusterRows)) {
+        st = launch_apply_cluster(p, x, y, rows, ld_x, ld_y, in_dtype, out_dtype, dir, stream);
+        if (st != HARP_ERR_UNSUPPORTED || choice == kCluster) return st;
         harp_clear_error();
     }
     if (choice == kAuto || choice == kTiled) {

@@ -286,11 +286,13 @@ __host__ __device__ __forceinline__ int stage_groups(int nb, int qv, int nthread
 // All items of one stage: items j = tid, tid + T, ...; item j is block c = j % nb of the
 // sub-tiles g = j / nb, g + G, ...  The block's coefficients are loaded into registers at
 // the start of the item (a second register buffer to prefetch the next block costs more
-// in register moves than it saves in latency at 8 warps per SM).
+// in register moves than it saves in latency at 8 warps per SM), except the first item's,
+// which the caller has already requested (prefetch_first) before the barrier that opens the
+// stage, so its L2 latency overlaps the barrier wait.
 template <int B, bool INV, int V, int NT>
 __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, const FastDiv& nbd,
                                           const FastDiv& sdv, typename VecOf<V>::T* tile, int d, int qv,
-                                          int mask) {
+                                          int mask, float (&w)[64]) {
     const int nb = d / B;
     const int G = stage_groups(nb, qv, NT);
     const int items = nb * G;
@@ -303,9 +305,8 @@ __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, c
     it.hi = sdv.div(it.c);
     it.lo = it.c - s * it.hi;
     const int dhi = sdv.div(NT), dlo = NT - s * dhi;
-    float w[64];
     for (int j = tid; j < items; j += NT) {
-        load_block<B>(w, sb, it.c);
+        if (j != tid) load_block<B>(w, sb, it.c);   // the first item's block is already requested
         apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, w);
         it.c += NT;
         it.lo += dlo;
@@ -322,6 +323,29 @@ __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, c
             it.hi = sdv.div(it.c);
             it.lo = it.c - s * it.hi;
         }
+    }
+}
+
+// Requests the block of this thread's first item of stage t (item j = tid) for a tile of qv
+// sub-tiles, into w; run_stage then uses it without loading it again.
+template <int MASK, int V, int NT>
+__device__ __forceinline__ void prefetch_first(const TiledParams& p, int t, int qv, int dl, uint32_t rank,
+                                               float (&w)[64]) {
+    const StageDesc& sd = p.pd.st[t];
+    const float* sb = p.lanes + p.lane_off[t] + (int64_t)rank * dl * sd.b;
+    const int tid = threadIdx.x;
+    switch (sd.b) {
+#define HARP_PREFETCH_CASE(RB)                                                                      \
+    case RB:                                                                                        \
+        if constexpr ((MASK >> RB) & 1) {                                                           \
+            const int nb = dl / RB;                                                                 \
+            if (tid < nb * stage_groups(nb, qv, NT)) load_block<RB>(w, sb, tid - nb * p.nb_div[t].div(tid)); \
+        }                                                                                           \
+        break;
+        HARP_PREFETCH_CASE(2) HARP_PREFETCH_CASE(3) HARP_PREFETCH_CASE(4) HARP_PREFETCH_CASE(5)
+        HARP_PREFETCH_CASE(6) HARP_PREFETCH_CASE(7) HARP_PREFETCH_CASE(8)
+#undef HARP_PREFETCH_CASE
+        default: break;
     }
 }
 
@@ -554,7 +578,11 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         __syncthreads();
         if (tid == 0) issue_tile<TIn>(p, t_idx, dl, col0, stage_buf, bar);
     }
-    // local stages in order: forward 0..m_local-1, inverse m_local-1..0
+    // local stages in order: forward 0..m_local-1, inverse m_local-1..0; each stage's first
+    // block is requested before the barrier that precedes the stage
+    float w[64];
+    const int t_first = INV ? m_local - 1 : 0;
+    prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_idx * R) + V - 1) / V), dl, rank, w);
     auto local_stages = [&](int qv) {
         for (int step = 0; step < m_local; ++step) {
             const int t = INV ? m_local - 1 - step : step;
@@ -566,13 +594,14 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
 #define HARP_TILED_CASE(RB)                                                                         \
     case RB:                                                                                        \
         if constexpr ((MASK >> RB) & 1)                                                             \
-            run_stage<RB, INV, V, NT>(sb, s, p.nb_div[t], p.s_div[t], tile, dl, qv, p.mask);       \
+            run_stage<RB, INV, V, NT>(sb, s, p.nb_div[t], p.s_div[t], tile, dl, qv, p.mask, w);    \
         break;
                 HARP_TILED_CASE(2) HARP_TILED_CASE(3) HARP_TILED_CASE(4) HARP_TILED_CASE(5)
                 HARP_TILED_CASE(6) HARP_TILED_CASE(7) HARP_TILED_CASE(8)
 #undef HARP_TILED_CASE
                 default: break;
             }
+            if (step + 1 < m_local) prefetch_first<MASK, V, NT>(p, INV ? t - 1 : t + 1, qv, dl, rank, w);
             __syncthreads();
         }
     };
@@ -616,6 +645,9 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         } else {
             local_stages(qv);
         }
+        if (t_next < p.ntiles)   // the next tile's first block, in flight during the drain and fill
+            prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_next * R) + V - 1) / V), dl,
+                                        rank, w);
         if constexpr (std::is_same<TOut, int8_t>::value)
             drain_tile_quant<V, NT>(tile, dl, nr, (int8_t*)p.y + row0 * p.ld_y, p.ld_y, p.mask,
                                     p.scales + row0 * p.ld_s, p.ld_s, p.qlanes);

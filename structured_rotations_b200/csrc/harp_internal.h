@@ -61,6 +61,7 @@ struct harp_plan_s {
     int8_t* d_signs = nullptr;
     int* d_status = nullptr;          // device error word (bounded waits)
     void* fast = nullptr;             // fast-path state (see apply_fast.cu)
+    void* cluster = nullptr;          // cluster-kernel split and table (see apply_cluster.cu)
     void* host_io = nullptr;          // streams and staging buffers of harp_apply_host (host_io.cu)
     std::mutex host_io_mu;            // harp_apply_host calls on this plan take turns
 };
@@ -99,6 +100,15 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
                               int64_t ld_x, int64_t ld_y, harp_dtype in_dtype, harp_dir dir,
                               void* stream, harp_dtype out_dtype);
 void fast_state_free(harp_plan_s* p);
+// Chooses the cluster kernel's split for plans it covers and builds their cluster table on
+// `stream` (apply_cluster.cu); a no-op for other plans, which then never take that kernel.
+void cluster_prepare(harp_plan_s* p, void* stream);
+void cluster_state_free(harp_plan_s* p);
+// Cluster row kernel (apply_cluster.cu): HARP_ERR_UNSUPPORTED for plans without a cluster
+// table, unaligned rows and fp32-in / bf16-out.
+harp_status launch_apply_cluster(const harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
+                                 int64_t ld_y, harp_dtype in_dtype, harp_dtype out_dtype, harp_dir dir,
+                                 void* stream);
 // Builds the specialized kernel's coefficient table (and its launch attributes) on
 // `stream` for plans it covers; a no-op for other plans.  Called by materialization, so
 // every later launch only reads the table.  A plan whose table cannot be built (no

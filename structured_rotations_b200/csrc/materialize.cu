@@ -123,6 +123,7 @@ harp_status harp_device_free(harp_plan_s* p) {
     cudaSetDevice(p->device);
     cudaDeviceSynchronize();
     fast_state_free(p);
+    cluster_state_free(p);
     host_io_free(p);
     cudaFree(p->d_blocks);
     cudaFree(p->d_blocks_lanes);
@@ -203,7 +204,8 @@ harp_status materialize_locked(harp_plan_s* p, void* stream_) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
-    fast_prepare(p, stream);   // the specialized kernel's table, so that launches only read plan state
+    fast_prepare(p, stream);      // the specialized kernel's table, so that launches only read plan state
+    cluster_prepare(p, stream);   // the cluster kernel's split and table
     e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     return HARP_OK;

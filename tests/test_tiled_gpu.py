@@ -128,10 +128,11 @@ def test_shapes_outside_the_tiled_kernel_fall_back(monkeypatch):
 
 
 def test_default_dispatch_takes_the_tiled_kernel_for_d5120_and_c5(monkeypatch):
+    """Batches of many rows (small ones take the cluster kernel, tests/test_cluster_gpu.py)."""
     monkeypatch.delenv("HARP_KERNEL", raising=False)
     for name, direction in (("d5120", "forward"), ("d8192_int8", "inverse"), ("d4096", "inverse")):
         gp, _ = plans(name)
-        run(gp, W.draw_encoded(W.get(name), 0, 64), direction)
+        run(gp, W.draw_encoded(W.get(name), 0, 1024), direction)
         assert H.last_kernel() == "harp_tiled_kernel", name
         gp.device_status()
 
