@@ -172,6 +172,24 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
     tp.staged_rows = (int)staged;
     tp.mask = (dl % 32 == 0) ? 0x18 : 0;
     tp.status = p->d_status;
+    // stages applied while filling / draining: radix 8 at stride 1, radix 2 at stride d / 2
+    // (whole rows in 4-row sub-tiles; the quantizer's drain keeps its stage).  Only when a tile
+    // is a single sub-tile (d = 8192: R = 4), where a pass over the tile is the largest share of
+    // the work: the fused fill and drain need 256 threads (more registers than a 384-thread CTA
+    // allows), which measured slower than the passes they save at d = 5120 (R = 8) and equal at
+    // d = 4096 (B200: d = 8192 forward 2.36 -> 2.12 ms, d = 5120 forward 1.24 -> 1.33 ms).
+    {
+        auto kind_of = [&](int t) {
+            const StageDesc& sd = pd.st[t];
+            if (sd.b == 8 && sd.s == 1) return (int)kFuseS1R8;
+            if (sd.b == 2 && 2 * sd.s == d) return (int)kFuseH2R2;
+            return (int)kFuseNone;
+        };
+        const bool can = sh.V == 4 && sh.R == 4 && cl == 1 && !std::getenv("HARP_TILED_NOFUSE");
+        const bool inv = dir == HARP_INVERSE;
+        tp.fuse_first = can ? kind_of(inv ? pd.m - 1 : 0) : kFuseNone;
+        tp.fuse_last = can && !quant && pd.m >= 2 ? kind_of(inv ? 0 : pd.m - 1) : kFuseNone;
+    }
     tp.wait_limit = g_inject_extra ? g_inject_limit : kWaitLimit;
     tp.extra_tx = g_inject_extra;
     tp.last_blocks = p->d_blocks + pd.st[pd.m - 1].block_off;
@@ -187,6 +205,8 @@ harp_status launch_apply_tiled(const harp_plan_s* p, const void* x, void* y, int
         const int qv = (int)((std::min<int64_t>(R, rows) + V - 1) / V);
         for (int t = 0; t < pd.m - (cl == 2 ? 1 : 0); ++t)
             if (stage_groups((int)(dl / pd.st[t].b), qv, kThreadChoices[1]) > 1) nt = kThreadChoices[0];
+        // the fused fill / drain need more than the 168 registers a 384-thread CTA allows
+        if (tp.fuse_first || tp.fuse_last) nt = kThreadChoices[0];
     }
     cudaStream_t s = (cudaStream_t)stream;
     const bool inv = dir == HARP_INVERSE;

@@ -71,6 +71,7 @@ struct TiledParams {
     float* scales;                     // quantized output (int8 codes in y): per-block scales
     int64_t ld_s;                      // scales per row of the scales array (row stride)
     int qlanes;                        // quantizer block / 8: lanes that hold one block
+    int fuse_first, fuse_last;         // stage applied while filling / draining the tile (kFuse*)
     long long wait_limit;              // polls of a staging wait before it gives up (kWaitLimit)
     uint32_t extra_tx;                 // test hook, normally 0: bytes each staging barrier is told to
                                        // expect beyond what is copied, so its first wait runs out
@@ -480,6 +481,158 @@ __device__ __forceinline__ void drain_tile(const typename VecOf<V>::T* tile, int
     }
 }
 
+// Stages applied while a tile is filled or drained (4-row sub-tiles), so they cost no pass of
+// their own over the tile in shared memory:
+//  kFuseS1R8  radix 8 at stride 1: the 8 consecutive coordinates a thread moves are one group
+//             (block c = the run's index);
+//  kFuseH2R2  radix 2 at stride d / 2: runs j and j + d / 16 hold the groups c = 8 j + e
+//             (coordinates c and c + d / 2).
+// The arithmetic is group_vec's: every output summed over its inputs in order from zero.
+enum { kFuseNone = 0, kFuseS1R8 = 1, kFuseH2R2 = 2 };
+
+// The 8 x 8 block c of a stage (lane-interleaved at sb; B, or B^T when TR) applied to 8 quads,
+// in two halves of four outputs so that only half of the block is in registers at a time:
+// outputs 4h .. 4h + 3 need rows 4h .. of B (pieces 8h .. 8h + 7 of the block) or columns
+// 4h .. of B (the first or second 16 bytes of each row: pieces 2l + h).
+template <bool TR>
+__device__ __forceinline__ void block8_quads(const float* __restrict__ sb, int c, const float4 (&xv)[8],
+                                             float4 (&yv)[8]) {
+    const float4* src = (const float4*)sb + (size_t)(c >> 5) * 16 * 32 + (c & 31);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldg(src + (TR ? 2 * i + h : 8 * h + i) * 32);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+        // forward: w[kk * 8 + l] = B[4h + kk][l]; inverse: w[l * 4 + kk] = B[l][4h + kk]
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) zero_v(yv[4 * h + kk]);
+#pragma unroll
+        for (int l = 0; l < 8; ++l)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) fma_v(yv[4 * h + kk], TR ? w[l * 4 + kk] : w[kk * 8 + l], xv[l]);
+    }
+}
+
+// One 2 x 2 block (stored B00, B01, B10, B11) applied to the quads of coordinates c and c + d/2.
+template <bool TR>
+__device__ __forceinline__ void block2_quads(const float4& wb, const float4& x0, const float4& x1, float4& y0,
+                                             float4& y1) {
+    const float w00 = wb.x, w01 = TR ? wb.z : wb.y, w10 = TR ? wb.y : wb.z, w11 = wb.w;
+    zero_v(y0);
+    zero_v(y1);
+    fma_v(y0, w00, x0);
+    fma_v(y0, w01, x1);
+    fma_v(y1, w10, x0);
+    fma_v(y1, w11, x1);
+}
+
+// fill_tile (4-row sub-tiles) with the stage `kind` applied on the way (blocks of that stage,
+// lane-interleaved, at sb; TR: transposed blocks, the inverse).
+template <int NT, typename TIn, bool TR>
+__device__ __forceinline__ void fill_tile_fused(float4* tile, int d, int nr, int n_staged, const TIn* staged,
+                                                const TIn* src, int64_t ld, int kind, const float* __restrict__ sb) {
+    auto row_ptr = [&](int r) -> const TIn* { return r < n_staged ? staged + (size_t)r * d : src + r * ld; };
+    auto load_rows = [&](const TIn* const (&rp)[4], int q, int col, float (&v)[4][8]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            load8(rp[e] + col, v[e]);
+            if (4 * q + e >= nr) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[e][k] = 0.0f;
+            }
+        }
+    };
+    for (int q = 0; 4 * q < nr; ++q) {
+        const TIn* rp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) rp[e] = row_ptr(min(4 * q + e, nr - 1));
+        float4* st = tile + q * d;
+        if (kind == kFuseS1R8) {
+            for (int j = threadIdx.x; j < d / 8; j += NT) {
+                float v[4][8];
+                load_rows(rp, q, 8 * j, v);
+                float4 xv[8], yv[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) xv[k] = make_float4(v[0][k], v[1][k], v[2][k], v[3][k]);
+                block8_quads<TR>(sb, j, xv, yv);
+                const int jx = j & 7;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) st[8 * j + (k ^ jx)] = yv[k];
+            }
+        } else {
+            const int h = d / 16;
+            for (int j = threadIdx.x; j < h; j += NT) {
+                float a[4][8], b[4][8];
+                load_rows(rp, q, 8 * j, a);
+                load_rows(rp, q, 8 * j + d / 2, b);
+                const int ja = j & 7, jb = (j + h) & 7;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 wb = __ldg((const float4*)sb + 8 * j + e);
+                    float4 y0, y1;
+                    block2_quads<TR>(wb, make_float4(a[0][e], a[1][e], a[2][e], a[3][e]),
+                                     make_float4(b[0][e], b[1][e], b[2][e], b[3][e]), y0, y1);
+                    st[8 * j + (e ^ ja)] = y0;
+                    st[8 * (j + h) + (e ^ jb)] = y1;
+                }
+            }
+        }
+    }
+}
+
+// 8 floats of row component e of 8 quads
+__device__ __forceinline__ void quad_lane(const float4 (&v4)[8], int e, float (&v)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = e == 0 ? v4[k].x : e == 1 ? v4[k].y : e == 2 ? v4[k].z : v4[k].w;
+}
+
+// drain_tile (4-row sub-tiles) with the stage `kind` applied on the way.
+template <int NT, typename TOut, bool TR>
+__device__ __forceinline__ void drain_tile_fused(const float4* tile, int d, int nr, TOut* dst, int64_t ld, int kind,
+                                                 const float* __restrict__ sb) {
+    for (int q = 0; 4 * q < nr; ++q) {
+        const float4* st = tile + q * d;
+        TOut* rp = dst + (4 * q) * ld;
+        const int rows = min(4, nr - 4 * q);
+        auto put = [&](const float4 (&y)[8], int col) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (e < rows) {
+                    quad_lane(y, e, v);
+                    store8(rp + e * ld + col, v);
+                }
+            }
+        };
+        if (kind == kFuseS1R8) {
+            for (int j = threadIdx.x; j < d / 8; j += NT) {
+                const int jx = j & 7;
+                float4 xv[8], yv[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) xv[k] = st[8 * j + (k ^ jx)];
+                block8_quads<TR>(sb, j, xv, yv);
+                put(yv, 8 * j);
+            }
+        } else {
+            const int h = d / 16;
+            for (int j = threadIdx.x; j < h; j += NT) {
+                const int ja = j & 7, jb = (j + h) & 7;
+                float4 y0[8], y1[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 wb = __ldg((const float4*)sb + 8 * j + e);
+                    block2_quads<TR>(wb, st[8 * j + (e ^ ja)], st[8 * (j + h) + (e ^ jb)], y0[e], y1[e]);
+                }
+                put(y0, 8 * j);
+                put(y1, 8 * j + d / 2);
+            }
+        }
+    }
+}
+
 // Fused quantizer epilogue (the rotated rows feed a blockwise quantizer, HARP technical
 // summary §2.4: a drop-in preprocessing step in front of the quantizer).  Each aligned
 // block of 8 qlanes coordinates of a row, with maximum magnitude a, becomes one fp32 scale
@@ -581,10 +734,21 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
     // local stages in order: forward 0..m_local-1, inverse m_local-1..0; each stage's first
     // block is requested before the barrier that precedes the stage
     float w[64];
-    const int t_first = INV ? m_local - 1 : 0;
-    prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_idx * R) + V - 1) / V), dl, rank, w);
+    // stages fused into the fill / drain (4-row sub-tiles of whole rows only) are not run here
+    const bool fused = V == 4 && CL == 1 && NT == 256;   // the launcher fuses only with 256 threads
+    const int step0 = fused && p.fuse_first ? 1 : 0;
+    const int step1 = m_local - (fused && p.fuse_last ? 1 : 0);
+    const int t_first = INV ? m_local - 1 - step0 : step0;
+    auto sb_of = [&](int t) { return p.lanes + p.lane_off[t] + (int64_t)rank * dl * p.pd.st[t].b; };
+    // Without fused stages the first block is requested early (before the loop, and before the
+    // drain of the previous tile), so its latency hides behind the drain and the fill; with them
+    // it is requested after the fill, whose fused stage needs the registers.
+    const bool early = !(fused && (p.fuse_first || p.fuse_last));
+    if (early && step0 < step1)
+        prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_idx * R) + V - 1) / V), dl, rank,
+                                    w);
     auto local_stages = [&](int qv) {
-        for (int step = 0; step < m_local; ++step) {
+        for (int step = step0; step < step1; ++step) {
             const int t = INV ? m_local - 1 - step : step;
             const StageDesc& sd = p.pd.st[t];
             // the slab's blocks of stage t start at block r dl / b_t
@@ -601,7 +765,7 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
 #undef HARP_TILED_CASE
                 default: break;
             }
-            if (step + 1 < m_local) prefetch_first<MASK, V, NT>(p, INV ? t - 1 : t + 1, qv, dl, rank, w);
+            if (step + 1 < step1) prefetch_first<MASK, V, NT>(p, INV ? t - 1 : t + 1, qv, dl, rank, w);
             __syncthreads();
         }
     };
@@ -628,8 +792,19 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
             }
             parity ^= 1;
         }
-        fill_tile<V, NT, TIn>(tile, dl, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x + col0,
-                              p.ld_x, p.mask);
+        if constexpr (V == 4 && CL == 1 && NT == 256) {
+            if (p.fuse_first)
+                fill_tile_fused<NT, TIn, INV>((float4*)tile, dl, nr, n_staged, (const TIn*)stage_buf,
+                                              (const TIn*)p.x + row0 * p.ld_x + col0, p.ld_x, p.fuse_first,
+                                              sb_of(INV ? m_local - 1 : 0));
+            else
+                fill_tile<V, NT, TIn>(tile, dl, nr, n_staged, (const TIn*)stage_buf,
+                                      (const TIn*)p.x + row0 * p.ld_x + col0, p.ld_x, p.mask);
+        } else {
+            fill_tile<V, NT, TIn>(tile, dl, nr, n_staged, (const TIn*)stage_buf, (const TIn*)p.x + row0 * p.ld_x + col0,
+                                  p.ld_x, p.mask);
+        }
+        if (!early && step0 < step1) prefetch_first<MASK, V, NT>(p, t_first, qv, dl, rank, w);
         __syncthreads();
         const int64_t t_next = t_idx + t_step;
         if (p.staged_rows && tid == 0 && t_next < p.ntiles && !failed) {
@@ -645,14 +820,21 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         } else {
             local_stages(qv);
         }
-        if (t_next < p.ntiles)   // the next tile's first block, in flight during the drain and fill
+        if (early && t_next < p.ntiles && step0 < step1)   // the next tile's, in flight during drain and fill
             prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_next * R) + V - 1) / V), dl,
                                         rank, w);
         if constexpr (std::is_same<TOut, int8_t>::value)
             drain_tile_quant<V, NT>(tile, dl, nr, (int8_t*)p.y + row0 * p.ld_y, p.ld_y, p.mask,
                                     p.scales + row0 * p.ld_s, p.ld_s, p.qlanes);
-        else
+        else if constexpr (V == 4 && CL == 1 && NT == 256) {
+            if (p.fuse_last)
+                drain_tile_fused<NT, TOut, INV>((const float4*)tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0,
+                                                p.ld_y, p.fuse_last, sb_of(INV ? 0 : m_local - 1));
+            else
+                drain_tile<V, NT, TOut>(tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0, p.ld_y, p.mask);
+        } else {
             drain_tile<V, NT, TOut>(tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0, p.ld_y, p.mask);
+        }
         __syncthreads();
     }
 }

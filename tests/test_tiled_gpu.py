@@ -183,3 +183,25 @@ def test_degenerate_and_large_radix_schedules(monkeypatch, schedule):
         out = run(gp, x, direction)
         check(out, tr.apply(xf, direction), xf, f"{schedule} {direction}")
     assert H.last_kernel() == "apply_simple_kernel"
+
+
+@pytest.mark.parametrize("schedule", [(8, 8, 8, 8, 2), (2, 8, 8, 8, 8, 2), (8, 4, 8, 8, 4)])
+@pytest.mark.parametrize("direction", ["forward", "inverse"])
+def test_stages_fused_into_fill_and_drain_match_separate_passes(monkeypatch, schedule, direction):
+    """At d = 8192 (a tile is one 4-row sub-tile) the radix-8 stride-1 stage and the radix-2
+    stride-d/2 stage run inside the tile's fill and drain; the result is the same, bit for bit,
+    as with every stage a pass of its own (HARP_TILED_NOFUSE=1), and matches the oracle."""
+    d = int(np.prod(schedule))
+    theta = W.draw_theta(O.theta_count(schedule), 0.2236, 77)
+    gp = H.Plan(d, schedule, theta=theta, sign_seed=78).materialize()
+    tr = O.Transform(O.make_plan(d, schedule, theta, sign_seed=78))
+    rng = np.random.default_rng(d + len(schedule))
+    enc = W.encode_bf16(rng.standard_normal((203, d)))
+    monkeypatch.setenv("HARP_KERNEL", "tiled")
+    a = run(gp, enc, direction)
+    monkeypatch.setenv("HARP_TILED_NOFUSE", "1")
+    b = run(gp, enc, direction)
+    assert np.array_equal(a, b)
+    xf = W.decode_bf16(enc)
+    check(a, tr.apply(xf, direction), xf, f"fused {schedule} {direction}")
+    gp.device_status()
