@@ -61,6 +61,9 @@ def parse_args():
     ap.add_argument("--grad-rows", type=int, default=0,
                     help="time only the calibration backward (harp_grad_theta) on this many d=4096 rows and "
                          "print its line (for profiling that kernel alone)")
+    ap.add_argument("--decode-rows", type=int, default=0,
+                    help="time only decode-shaped calls (this many rows of the d=8192 int8 workload, forward) "
+                         "and print their line (for profiling that call alone)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--rows", type=int, default=0, help="rows per GPU (default: the workload's; "
@@ -639,6 +642,18 @@ def run_ours(args):
                                  device_id=device)
         dist = tdist
 
+    if args.decode_rows:
+        wd = W.get("d8192_int8")
+        pd_ = make_plan("d8192_int8", H, W)
+        xd = to_device_bf16(W.draw_encoded(wd, 0, args.decode_rows), torch, device)
+        yd = torch.empty_like(xd)
+        dev_us, host_us, wall_us, kn = time_calls(pd_, xd, yd, max(1, args.steps), max(3, args.warmup), torch,
+                                                  "forward")
+        pd_.device_status()
+        print(json.dumps({"workload": f"d=8192 schedule (8,8,8,8,2), int8 theta, {args.decode_rows} bf16 rows, "
+                                      "forward", "device_us_per_call": dev_us, "host_us_per_call": host_us,
+                          "us_per_call": wall_us, "kernel": kn}))
+        return 0
     if args.quant_rows:
         peak, _ = peaks()
         print(json.dumps(quant_measurement(args, H, W, torch, device, peak, rows=args.quant_rows)))

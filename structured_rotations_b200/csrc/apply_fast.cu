@@ -72,17 +72,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// Two values split into x = hi + lo for the three-product TF32 scheme.  hi is x rounded to
-// 11 significant bits (ties away from zero) by integer arithmetic on its bit pattern: add
-// half of bit 13, clear bits 0-12 (a carry into the exponent is the correct rounding), so
-// hi is exact in TF32; lo = x - hi is exact in fp32 (at most 13 significant bits), and the
-// tensor core reads its top 11, so |x - hi - lo_tf32| <= 2^-22 |x|.  The rounding runs on
-// the integer ALU pipe and only the subtraction on the FMA pipe, which the tensor-core
-// stages keep busy otherwise.  Valid for finite x below the largest binade.
+// Two values split into x = hi + lo for the three-product TF32 scheme.  hi is x truncated to
+// 11 significant bits (bits 0-12 of the pattern cleared, one logic instruction), so hi is
+// exact in TF32 and |lo| < 2^-10 |x|; lo = x - hi is exact in fp32 (at most 13 significant
+// bits), and the tensor core reads its top 11, so |x - hi - lo_tf32| < 2^-21 |x|.  The
+// dropped product lo_a lo_b is below 2^-20 |a b|.  Only the subtraction uses the FMA pipe.
 __device__ __forceinline__ void split2_tf32(float a, float b, uint32_t& ha, uint32_t& hb, uint32_t& la,
                                             uint32_t& lb) {
-    ha = (__float_as_uint(a) + 0x1000u) & 0xffffe000u;
-    hb = (__float_as_uint(b) + 0x1000u) & 0xffffe000u;
+    ha = __float_as_uint(a) & 0xffffe000u;
+    hb = __float_as_uint(b) & 0xffffe000u;
     la = __float_as_uint(__fsub_rn(a, __uint_as_float(ha)));
     lb = __float_as_uint(__fsub_rn(b, __uint_as_float(hb)));
 }
