@@ -54,7 +54,10 @@ differences, one-stage closed forms, stationarity, additivity), the blockwise in
 quantizer of the rotated rows (§2.4; tests/test_oracle_quant_pins.py: hand-worked
 codes, zero blocks, the half-step bound, scaling) and the composition of rotations
 (tests/test_oracle_compose_pins.py: the theta = 0 product of signed Hadamards,
-orthogonality, inverse, factor order).
+orthogonality, inverse, factor order).  The fit's evaluation terms R_bd and L_diag
+(tests/test_oracle_fit_pins.py: invariants and closed forms only) and the moment check that
+picks the number of composed passes (tests/test_oracle_moment_pins.py: one-hot and flat
+rows, scale invariance, Hoelder bounds, a one-hot row flattened by one theta = 0 pass).
 """
 from __future__ import annotations
 
@@ -549,3 +552,46 @@ def l_diag(w_rot: np.ndarray, h_rot: np.ndarray, q: int) -> float:
     codes, scales = quantize_blocks(w, q)
     target = (codes.reshape(w.shape[0], -1, q) * scales[..., None]).reshape(w.shape)
     return float(np.sum(np.diag(h_rot)[None, :] * (w - target) ** 2))
+
+
+# ---------------------------------------------------------------------------
+# Moment check that picks the number of composed passes
+# ---------------------------------------------------------------------------
+#
+# The RHT-composition page proposes a linear-time check on the input's moments that adapts at
+# run time how many randomized Hadamard passes are applied, without giving the statistic or
+# its thresholds.  Reading: one pass turns x into coordinates that are Rademacher-weighted sums
+# of the entries of x, whose distance from a Gaussian is governed by how concentrated x is;
+# the check computes, per row, the moments
+#     m2 = sum x_i^2,  m3 = sum |x_i|^3,  m4 = sum x_i^4
+# and from them the Berry-Esseen ratio rho = m3 / m2^(3/2) (in [d^-1/2, 1]) and the peakedness
+# kappa = m4 / m2^2 (in [1/d, 1]: 1/d for a flat row, 1 for a one-hot row).  The number of
+# passes is the smallest k in (1, 2, 3) whose threshold the row meets: kappa <= tau_1 -> 1,
+# kappa <= tau_2 -> 2, else 3 (three for block (vector) quantizers in any case, per the page);
+# the thresholds are the caller's.
+
+def row_moments(x: np.ndarray) -> np.ndarray:
+    """[rows, 3] float64: (sum x^2, sum |x|^3, sum x^4) of every row."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    return np.stack([np.sum(a * a, axis=1), np.sum(a * a * a, axis=1), np.sum((a * a) * (a * a), axis=1)], axis=1)
+
+
+def peakedness(m: np.ndarray) -> np.ndarray:
+    """kappa = m4 / m2^2 per row (0 for a zero row)."""
+    m = np.asarray(m, dtype=np.float64)
+    m2 = m[:, 0]
+    return np.where(m2 > 0, m[:, 2] / np.where(m2 > 0, m2 * m2, 1.0), 0.0)
+
+
+def berry_esseen_ratio(m: np.ndarray) -> np.ndarray:
+    """rho = m3 / m2^(3/2) per row (0 for a zero row)."""
+    m = np.asarray(m, dtype=np.float64)
+    m2 = m[:, 0]
+    return np.where(m2 > 0, m[:, 1] / np.where(m2 > 0, m2 ** 1.5, 1.0), 0.0)
+
+
+def passes_needed(kappa: np.ndarray, tau1: float, tau2: float) -> np.ndarray:
+    """The smallest number of passes (1, 2 or 3) whose threshold each row's kappa meets."""
+    kappa = np.asarray(kappa, dtype=np.float64)
+    return np.where(kappa <= tau1, 1, np.where(kappa <= tau2, 2, 3)).astype(np.int32)
