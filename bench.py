@@ -464,7 +464,36 @@ def side_measurements(args, H, W, torch, device, peak):
     del wt, wo, ws
     out.append(quant_measurement(args, H, W, torch, device, peak))
     out.append(compose_measurement(args, H, W, torch, device, peak))
+    out.append(moment_measurement(args, H, W, torch, device, peak))
     return out
+
+
+def moment_measurement(args, H, W, torch, device, peak, steps=20):
+    """The moment check that picks the number of composed passes (harp_moment_check) on the
+    d = 4096 workload's rows: one read of the rows (2 d bytes each), per-row moments and pass
+    counts written (28 bytes each)."""
+    w = W.get("d4096")
+    x = to_device_bf16(W.draw_encoded(w, 0, w.rows), torch, device)
+    m = torch.empty(w.rows, 3, dtype=torch.float64, device=device)
+    k = torch.empty(w.rows, dtype=torch.int32, device=device)
+    tau1, tau2 = 4.0 / w.d, 40.0 / w.d
+    for _ in range(3):
+        H.moment_check(x, tau1, tau2, m, k)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        H.moment_check(x, tau1, tau2, m, k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    byt = w.rows * (2 * w.d + 28)
+    counts = torch.bincount(k, minlength=4).cpu().tolist()
+    return {"workload": f"moment check (passes for tau = 4/d, 40/d): d=4096, {w.rows} bf16 rows", "kernel_ms": ms,
+            "rows_per_s": w.rows / (ms / 1e3), "hbm_gbs": byt / (ms / 1e3) / 1e9,
+            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": "moment_check_kernel",
+            "rows_needing_1_2_3_passes": counts[1:4]}
 
 
 def fit_measurement(H, W, torch, device, peak, pv, w_rot, w4, q=128, steps=10):

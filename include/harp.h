@@ -348,6 +348,25 @@ HARP_API harp_status harp_l_diag(const void* w, int64_t rows, int64_t cols, int6
                                  const float* h, int64_t ld_h, int32_t qblock, double* out, void* stream);
 
 /*
+ * harp_moment_check — the check that picks how many composed passes a batch needs (the
+ * RHT-composition results quoted with the HARP pages propose a linear-time check on the
+ * input's moments that adapts the number of randomized Hadamard passes at run time, without
+ * giving the statistic or its thresholds).  Per row r of x:
+ *   moments[3r .. 3r+2] = (sum x^2, sum |x|^3, sum x^4)          (double)
+ *   passes[r] = 1 if kappa <= tau1, 2 if kappa <= tau2, else 3,   kappa = m4 / m2^2
+ * kappa is 1/d for a flat row and 1 for a one-hot row (0 for a zero row, which takes 1 pass);
+ * the Berry-Esseen ratio m3 / m2^1.5 follows from the moments.  Compose that many plans
+ * (harp_plan_compose) for the batch.
+ *   x         device rows, element type dtype, leading dimension ld >= d.
+ *   moments   device double array of 3 rows entries, or NULL.
+ *   passes    device int32 array of rows entries, or NULL (not both NULL).
+ * tau1 <= tau2, else HARP_ERR_INVALID_ARG; the outputs must not overlap x or each other.
+ * rows = 0 is a no-op.  Asynchronous on `stream`.
+ */
+HARP_API harp_status harp_moment_check(const void* x, int64_t rows, int64_t d, int64_t ld, harp_dtype dtype,
+                                       double tau1, double tau2, double* moments, int32_t* passes, void* stream);
+
+/*
  * harp_plan_compose — one plan for the composition T = T_{k-1} ... T_1 T_0 of k plans of
  * the same dimension (plans[0] acts first): k independent rotations in one pass over the
  * rows (composing two or three randomized Hadamard transforms brings every input's

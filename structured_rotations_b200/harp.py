@@ -82,6 +82,8 @@ def lib():
         "harp_off_block_energy": (_c_i32, [_vp, _c_i64, _c_i64, _c_i32, _c_i32, _vp, _vp]),
         "harp_l_diag": (_c_i32, [_vp, _c_i64, _c_i64, _c_i64, _c_i32, _vp, _c_i64, _c_i32, _vp, _vp]),
         "harp_test_inject_wait_timeout": (_c_i32, [_c_i64, ctypes.c_uint32]),
+        "harp_moment_check": (_c_i32, [_vp, _c_i64, _c_i64, _c_i64, _c_i32, ctypes.c_double, ctypes.c_double, _vp,
+                                       _vp, _vp]),
         "harp_plan_destroy": (_c_i32, [_vp]),
         "harp_status_string": (ctypes.c_char_p, [_c_i32]),
         "harp_last_error": (ctypes.c_char_p, []),
@@ -411,3 +413,19 @@ def inject_wait_timeout(poll_limit: int = 0, extra_bytes: int = 0) -> None:
     """Test hook (harp_test_inject_wait_timeout): make the staging waits of this thread's
     next tiled-kernel launches run out after poll_limit polls; (0, 0) clears it."""
     _check(lib().harp_test_inject_wait_timeout(poll_limit, extra_bytes), "harp_test_inject_wait_timeout")
+
+
+def moment_check(x, tau1: float = 0.0, tau2: float = 0.0, moments=None, passes=None, stream=None):
+    """Per row of the device rows x (harp_moment_check): (sum x^2, sum |x|^3, sum x^4) as a float64
+    tensor [rows, 3], and the number of composed passes (1 if m4 / m2^2 <= tau1, 2 if <= tau2, else
+    3) as an int32 tensor [rows].  Returns (moments, passes)."""
+    import torch
+    rows, d = x.shape
+    if moments is None:
+        moments = torch.empty(rows, 3, dtype=torch.float64, device=x.device)
+    if passes is None:
+        passes = torch.empty(rows, dtype=torch.int32, device=x.device)
+    _check(lib().harp_moment_check(x.data_ptr(), rows, d, _ld(x), _dtype_code(x), float(tau1), float(tau2),
+                                   moments.data_ptr(), passes.data_ptr(), _stream_handle(stream)),
+           "harp_moment_check")
+    return moments, passes

@@ -217,3 +217,17 @@ def test_fit_term_argument_errors_before_any_device_call():
     assert L.harp_l_diag(p, 4, 512, 512, HB.HARP_F32, p, 511, 32, out, None) == HB.HARP_ERR_INVALID_ARG
     assert L.harp_l_diag(p, 4, 512, 512, HB.HARP_F32, None, 512, 32, out, None) == HB.HARP_ERR_INVALID_ARG
     assert L.harp_l_diag(p, 4, 512, 512, 3, p, 512, 32, out, None) == HB.HARP_ERR_UNSUPPORTED
+
+
+def test_moment_check_argument_errors_before_any_device_call():
+    L = H.lib()
+    p = ctypes.c_void_p(16)
+    out = ctypes.c_void_p(1 << 40)
+    assert L.harp_moment_check(p, 4, 64, 64, 7, 0.1, 0.2, out, None, None) == HB.HARP_ERR_UNSUPPORTED
+    assert L.harp_moment_check(p, -1, 64, 64, HB.HARP_F32, 0.1, 0.2, out, None, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_moment_check(p, 4, 64, 63, HB.HARP_F32, 0.1, 0.2, out, None, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_moment_check(p, 4, 64, 64, HB.HARP_F32, 0.3, 0.2, out, None, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_moment_check(p, 4, 64, 64, HB.HARP_F32, 0.1, 0.2, None, None, None) == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_moment_check(p, 4, 64, 64, HB.HARP_F32, 0.1, 0.2, ctypes.c_void_p(32), None, None) \
+        == HB.HARP_ERR_INVALID_ARG
+    assert L.harp_moment_check(None, 0, 64, 64, HB.HARP_F32, 0.1, 0.2, None, None, None) == HB.HARP_OK
