@@ -595,11 +595,12 @@ def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):
     torch.cuda.synchronize()
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     byt = w.rows * (2 * w.d + w.d + 4 * (w.d // qblock))
+    kn = H.last_kernel()
     return {"workload": f"rotate + int8 quantize (qblock {qblock}): d=4096 schedule (8,8,8,8), {w.rows} bf16 rows "
                         f"-> int8 codes + fp32 scales, forward",
             "kernel_ms": ms, "rows_per_s": w.rows / (ms / 1e3), "hbm_gbs": byt / (ms / 1e3) / 1e9,
-            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": H.last_kernel() + " (int8 epilogue)",
-            "traffic": recorded_traffic("harp_tiled_kernel", "quant_d4096") if rows is None else None}
+            "hbm_frac": byt / (ms / 1e3) / 1e9 / peak, "kernel": kn + " (int8 epilogue)",
+            "traffic": recorded_traffic(kn, "quant_d4096") if rows is None else None}
 
 
 def grad_roofline(res, clocks, device, torch):

@@ -193,7 +193,8 @@ HARP_API harp_status harp_apply_host(harp_plan_t plan, const void* x, void* y, i
  *   q        device int8 codes, rows of d, leading dimension ld_q >= d.
  *   scales   device float, rows of d / qblock scales, leading dimension ld_s >= d / qblock.
  *   qblock   32, 64, 128 or 256, dividing d; else HARP_ERR_INVALID_ARG.
- * x, q and scales must not overlap.  Runs on the general tiled kernel: radices <= 8,
+ * x, q and scales must not overlap.  Runs on the specialized d = 4096 (8,8,8,8) kernel for
+ * that schedule, forward, from 32 rows up, else on the general tiled kernel: radices <= 8,
  * d % 8 == 0, x and q rows 16-byte aligned (ld_q a multiple of 16), scales 4-byte aligned;
  * otherwise HARP_ERR_UNSUPPORTED.  rows = 0 is a no-op.  Asynchronous on `stream`.
  */

@@ -159,6 +159,12 @@ extern "C" harp_status harp_apply_quant(harp_plan_t p, const void* x, int64_t ro
                  sb = ((rows - 1) * ld_s + d / qblock) * sizeof(float);
     if (ranges_overlap(x, xb, q, qb) || ranges_overlap(x, xb, scales, sb) || ranges_overlap(q, qb, scales, sb))
         return harp_fail(HARP_ERR_INVALID_ARG, "x, q and scales overlap");
+    const int choice = kernel_choice();
+    if (choice == kAuto || choice == kFast) {
+        st = launch_apply_fast_quant(p, x, rows, ld_x, q, ld_q, scales, ld_s, qblock, dir, stream);
+        if (st != HARP_ERR_UNSUPPORTED || choice == kFast) return st;
+        harp_clear_error();
+    }
     QuantOut qo{scales, ld_s, qblock};
     st = launch_apply_tiled(p, x, q, rows, ld_x, ld_q, HARP_BF16, HARP_BF16, dir, stream, &qo);
     if (st == HARP_ERR_UNSUPPORTED)

@@ -54,7 +54,7 @@ constexpr int kHalfBytes = kSFloats * 4;     // 65536
 constexpr int kXBytes = 16 * 128;            // one 16-row x 64-column bf16 input box per warp
 constexpr int kXOffset = (kEFloats + kSFloats) * 4;          // 196608, 1024-aligned
 constexpr int kBarOffset = kXOffset + kWarps * kXBytes;      // 229376
-constexpr size_t kSmemBytes = (size_t)kBarOffset + 8 * (kWarps + 1) + 16 + 1024;   // + TMEM slot, alignment slack
+constexpr size_t kSmemBytes = (size_t)kBarOffset + 8 * (kWarps + 2) + 16 + 1024;   // + TMEM slot, alignment slack
 constexpr int kTmemCols = 512;               // the SM's whole tensor memory: 128 columns per warp
 constexpr long long kWaitLimit = 1ll << 26;  // mbarrier polls before giving up
 
@@ -64,6 +64,10 @@ struct FastParams {
     int ntiles;
     const float4* frag;      // B fragments, [cta rank][warp][column / 4][lane] float4 (see pack kernel)
     int* status;
+    int8_t* q;               // quantizing variant: int8 codes, rows of 4096, leading dimension ldq
+    int64_t ldq;
+    float* scales;           // and one scale per block of QB coordinates, leading dimension lds
+    int64_t lds;
 };
 
 // ----------------------------------------------------------------- PTX ---
@@ -163,21 +167,33 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 //
 // E[half][beta_local][row][pos]: half = beta >> 5 (the CTA whose chunks produced it),
 // beta_local = beta & 31, a_local = pencil index inside the owning CTA (a = 32 r + a_local)
-// and pos = a_local ^ swz(row, beta) with swz = (row & 7) | ((beta & 3) << 3).
+// and pos = a_local ^ swz(row, beta), swz = (row & 7) | (c(beta) << 3) with c = beta & 3 in
+// the bf16 variant and c = (beta ^ (beta >> 4)) & 3 in the quantizing one.
 //  - phase A stores one scalar per lane with beta fixed, row = g (+8) and a_local = l + 8q:
 //    (l + 8q) ^ (g + 8c) has l ^ g in bits 0-2 and q ^ c in bits 3-4, 32 banks.
 //  - phase B loads one scalar per lane with a_local fixed, row = g (+8) and
-//    beta = q + 8m (+4), so beta & 3 = q: a_local ^ (g + 8q), 32 banks.
+//    beta = q + 8m (+4), so beta & 3 = q and (beta >> 4) & 3 = m >> 1 for the whole
+//    instruction: a_local ^ (g + 8 (q ^ const)), 32 banks.
+//  - the quantizing variant also stores its outputs back in place (a_local fixed, row = g (+8),
+//    beta = l + 16q + 8e for fixed l, e: beta & 3 = l & 3, (beta >> 4) & 3 = q), which the
+//    (beta >> 4) term spreads: a_local ^ (g + 8 ((l & 3) ^ q)), 32 banks; its epilogue reads a
+//    row with lane = a_local and beta fixed, a permutation of one 32-float run.
 // Each chunk's 16 x 32 block is contiguous (2 KB), so the part of it bound for the partner
 // CTA is sent with one bulk copy as soon as the warp has produced it.
-__device__ __forceinline__ int e_index(int half, int row, int a_local, int beta) {
-    const int swz = (row & 7) | ((beta & 3) << 3);
-    return ((half * 32 + (beta & 31)) * 16 + row) * 32 + (a_local ^ swz);
+template <int QB>
+__device__ __forceinline__ int swz_of(int row, int beta) {
+    if constexpr (QB == 0) return (row & 7) | ((beta & 3) << 3);
+    else return (row & 7) | (((beta ^ (beta >> 4)) & 3) << 3);
 }
 
+template <int QB>
+__device__ __forceinline__ int e_index(int half, int row, int a_local, int beta) {
+    return ((half * 32 + (beta & 31)) * 16 + row) * 32 + (a_local ^ swz_of<QB>(row, beta));
+}
+
+template <int QB>
 __device__ __forceinline__ int s_index(int row, int a_local, int beta) {
-    const int swz = (row & 7) | ((beta & 3) << 3);
-    return ((beta & 31) * 16 + row) * 32 + (a_local ^ swz);
+    return ((beta & 31) * 16 + row) * 32 + (a_local ^ swz_of<QB>(row, beta));
 }
 
 // Output staging O[row][a_local][beta] (bf16), stored in 16-byte chunks of 8 beta values
@@ -348,8 +364,119 @@ __device__ __forceinline__ void store_row(const unsigned char* O, const FastPara
     }
 }
 
+// ------------------------------------------------- quantizing epilogue ---
+//
+// The quantizing variant (QB = 32, 64, 128 or 256, the blockwise int8 quantizer of the fused
+// rotate-then-quantize call) leaves each fp32 output in E where phase B read its input (see
+// e_index), then warp w quantizes row w of the tile:
+//  - lane L holds pencil a_local = L of the row for all 64 beta (64 conflict-free loads); a
+//    block of QB coordinates is, in this CTA's view, the pencils of beta >> SH (QB >= 64: the
+//    other 32 pencils are the partner's) or of one beta (QB = 32: the block is this CTA's);
+//  - block maxima: |y| maximised over the lane's beta of the block, then over the warp
+//    (redux.sync on the fp32 bit patterns, which order like the values for |y| >= 0);
+//  - QB >= 64: lane kb sends block kb's maximum to the partner's AMX[w][kb] (st.async,
+//    completed on the partner's qbar) and takes the larger of its own and the partner's;
+//  - s = a / 127 and 127 / a (fp32, round to nearest; 0 for a = 0) for the lane's blocks,
+//    the reciprocals passed round by shuffles; codes clamp(rne(y * (127 / a)), -127, 127)
+//    go byte by byte into the 32-byte runs CS[w][beta] and leave as 16-byte stores (the run
+//    of beta holds coordinates 64 beta + 32 r .. + 31).
+// S holds AMX (4 KB) and CS (32 KB) here: S is free from phase B (the partner has
+// received this CTA's chunks) until the next tile's phase A, which starts only after every
+// thread of both CTAs has passed this epilogue (the tile-end cluster barrier).
+constexpr int kAmxOffset = 0, kCsOffset = 4096;
+
+// round to nearest even, saturated to [-128, 127]
+__device__ __forceinline__ uint32_t cvt_rni_sat_s8(float x) {
+    uint32_t r;
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(remote_bar)
+                 : "memory");
+}
+
+template <int QB>
+__device__ __forceinline__ void quant_row(const float* E, unsigned char* S, const FastParams& p, int64_t row0, int r,
+                                          int w, int lane, uint64_t* qbar, uint32_t qparity, uint32_t remote_s,
+                                          uint32_t remote_qbar) {
+    constexpr int SH = QB <= 64 ? 0 : (QB == 128 ? 1 : 2);   // block of beta >> SH
+    constexpr int NLOC = 64 >> SH;                           // blocks of the row in this CTA's view
+    constexpr bool XCH = QB >= 64;                           // blocks span both CTAs
+    float v[64];
+#pragma unroll
+    for (int beta = 0; beta < 64; ++beta) v[beta] = E[e_index<QB>(beta >> 5, w, lane, beta)];
+    float own0 = 0.f, own1 = 0.f;   // lane L: the maxima of blocks L and L + 32
+#pragma unroll
+    for (int kb = 0; kb < NLOC; ++kb) {
+        float m = 0.f;
+#pragma unroll
+        for (int t = 0; t < (1 << SH); ++t) m = fmaxf(m, fabsf(v[(kb << SH) + t]));
+        const float wm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+        if (kb < 32) own0 = lane == kb ? wm : own0;
+        else own1 = lane == kb - 32 ? wm : own1;
+    }
+    float a0 = own0, a1 = own1;
+    if constexpr (XCH) {
+        const uint32_t dst = remote_s + kAmxOffset + (uint32_t)(w * 64 + lane) * 4u;
+        if (lane < NLOC) st_async_b32(dst, __float_as_uint(own0), remote_qbar);
+        if (NLOC > 32) st_async_b32(dst + 128u, __float_as_uint(own1), remote_qbar);
+        if (!mbar_wait(qbar, qparity)) {
+            if (lane == 0) atomicExch(p.status, 1);
+            mbar_wait(qbar, qparity);   // bounded again: no store may land after exit
+        }
+        const float* amx = reinterpret_cast<const float*>(S + kAmxOffset) + w * 64;
+        if (lane < NLOC) a0 = fmaxf(own0, amx[lane]);
+        if (NLOC > 32) a1 = fmaxf(own1, amx[lane + 32]);
+    }
+    float inv0 = 0.f, inv1 = 0.f;   // lane L: 127 / a of blocks L and L + 32
+    const int64_t grow = row0 + w;
+#pragma unroll
+    for (int h = 0; h < (NLOC > 32 ? 2 : 1); ++h) {
+        const int kb = lane + 32 * h;
+        if (kb < NLOC) {
+            const float a = h ? a1 : a0;
+            const float iv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+            if (h) inv1 = iv;
+            else inv0 = iv;
+            if (grow < p.rows) {
+                if constexpr (XCH) {
+                    if (r == 0) p.scales[grow * p.lds + kb] = __fdiv_rn(a, 127.f);
+                } else {
+                    p.scales[grow * p.lds + 2 * kb + r] = __fdiv_rn(a, 127.f);   // block (beta = kb, CTA r)
+                }
+            }
+        }
+    }
+    // Codes: |y| <= a gives |y * fl(127 / a)| <= 127 (1 + 2^-23), so the round-to-nearest
+    // conversion lands in [-127, 127]; the saturating conversion to s8 keeps that bound
+    // without a separate clamp.
+    unsigned char* cs = S + kCsOffset + w * 2048;
+#pragma unroll
+    for (int kb = 0; kb < NLOC; ++kb) {
+        const float iv = __shfl_sync(0xffffffffu, kb < 32 ? inv0 : inv1, kb & 31);
+#pragma unroll
+        for (int t = 0; t < (1 << SH); ++t) {
+            const int beta = (kb << SH) + t;
+            cs[beta * 32 + lane] = (unsigned char)(cvt_rni_sat_s8(v[beta] * iv) & 0xffu);
+        }
+    }
+    __syncwarp();
+    if (grow < p.rows) {
+        // runs beta = 2 lane and 2 lane + 1: 64 contiguous staging bytes, two 32-byte runs out
+        const uint4* src = reinterpret_cast<const uint4*>(cs + 64 * lane);
+        int8_t* dst = p.q + grow * p.ldq + 32 * r + 128 * lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(dst + 64 * (k >> 1) + 16 * (k & 1)) = src[k];
+    }
+}
+
 // ------------------------------------------------------------- kernel ---
 
+// QB = 0: bf16 rows out.  QB = 32 .. 256: int8 codes and per-block scales out (quant_row).
+template <int QB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     harp_fast_d4096_fwd_kernel(const __grid_constant__ CUtensorMap tmap_x, FastParams p) {
     extern __shared__ unsigned char smem_raw[];
@@ -361,7 +488,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     unsigned char* X = base + kXOffset;
     uint64_t* xbar = reinterpret_cast<uint64_t*>(base + kBarOffset);   // one per warp
     uint64_t* bar = xbar + kWarps;                                      // exchange
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+    uint64_t* qbar = bar + 1;                                           // partner's block maxima
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -372,7 +500,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     // tensor memory: the whole 512 columns; warp w uses lanes 32 (w & 3).., columns 128 (w >> 2)..
     if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
-    if (tid == 0) mbar_init(bar, 1);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(qbar, 1);
+    }
     if (lane == 0) mbar_init(xbar + warp, 1);
     tmem_fence_before_sync();
     __syncthreads();
@@ -399,6 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const uint32_t remote_e = map_to_rank(smem_u32(E + r * kSFloats), (uint32_t)(r ^ 1));   // partner's half r
     const uint32_t remote_bar = map_to_rank(smem_u32(bar), (uint32_t)(r ^ 1));
+    const uint32_t remote_s = map_to_rank(smem_u32(S), (uint32_t)(r ^ 1));
+    const uint32_t remote_qbar = map_to_rank(smem_u32(qbar), (uint32_t)(r ^ 1));
     cluster_arrive();
     cluster_wait();     // barriers initialised on both CTAs
     cluster_arrive();   // "my E may be written": matched by the wait at the top of the first tile
@@ -408,12 +541,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(xbar + warp, kXBytes);
         tma_load_2d(Xw, &tmap_x, 64 * (32 * r + 2 * warp), pair * kTile, xbar + warp);
     }
-    uint32_t xparity = 0, parity = 0;
+    uint32_t xparity = 0, parity = 0, qparity = 0;
     int64_t prev_row0 = -1;           // tile whose output still sits in O
 
     for (int tile = pair; tile < p.ntiles; tile += npairs) {
         const int64_t row0 = (int64_t)tile * kTile;
-        if (tid == 0) mbar_arrive_expect_tx(bar, kHalfBytes);
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, kHalfBytes);
+            // the partner's block maxima of this tile (16 rows of 4096 / QB blocks)
+            if constexpr (QB >= 64) mbar_arrive_expect_tx(qbar, 16u * (4096u / QB) * 4u);
+        }
 
         // -------------------------------------------------- phase A ---
 #pragma unroll 1
@@ -466,7 +603,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (task == 0) {
                 // row `warp` of the previous tile's output leaves O, which aliases the part
                 // of S this warp is about to write
-                if (prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
+                if (QB == 0 && prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
                 __syncwarp();
                 cluster_wait();       // the partner has finished reading its E (previous tile)
             }
@@ -477,11 +614,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int hh = 0; hh < 2; ++hh) {   // hh = destination CTA
                     const float va = y1[l][hh], vb = y1[l][hh + 2];
                     if (hh == r) {
-                        E[e_index(r, g, a_local, beta)] = va;
-                        E[e_index(r, g + 8, a_local, beta)] = vb;
+                        E[e_index<QB>(r, g, a_local, beta)] = va;
+                        E[e_index<QB>(r, g + 8, a_local, beta)] = vb;
                     } else {
-                        S[s_index(g, a_local, beta)] = va;
-                        S[s_index(g + 8, a_local, beta)] = vb;
+                        S[s_index<QB>(g, a_local, beta)] = va;
+                        S[s_index<QB>(g + 8, a_local, beta)] = vb;
                     }
                 }
             }
@@ -513,10 +650,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int m = 0; m < 8; ++m) {
                 const int half = m >> 2;
                 const int b0 = q + 8 * m, b1 = q + 4 + 8 * m;
-                v2[m][0] = E[e_index(half, g, a_local, b0)];
-                v2[m][1] = E[e_index(half, g + 8, a_local, b0)];
-                v2[m][2] = E[e_index(half, g, a_local, b1)];
-                v2[m][3] = E[e_index(half, g + 8, a_local, b1)];
+                v2[m][0] = E[e_index<QB>(half, g, a_local, b0)];
+                v2[m][1] = E[e_index<QB>(half, g + 8, a_local, b0)];
+                v2[m][2] = E[e_index<QB>(half, g, a_local, b1)];
+                v2[m][3] = E[e_index<QB>(half, g + 8, a_local, b1)];
             }
             tmem_wait_ld();
             float zz2[8][4];
@@ -529,24 +666,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             float y3[8][4];
             mma_stage_f32(a3, bw, y3);
             if (task == 0) cluster_wait();   // my copies have landed too: O (= S) may be written
-            // bf16 runs of 8 consecutive beta (i2 = 0..7) for i3 = 2q + e, rows g and g + 8
+            if constexpr (QB == 0) {
+                // bf16 runs of 8 consecutive beta (i2 = 0..7) for i3 = 2q + e, rows g and g + 8
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
+                for (int e = 0; e < 2; ++e) {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int c = e + 2 * hh;
-                    const uint4 pk = make_uint4(pack_bf16x2(y3[0][c], y3[1][c]), pack_bf16x2(y3[2][c], y3[3][c]),
-                                                pack_bf16x2(y3[4][c], y3[5][c]), pack_bf16x2(y3[6][c], y3[7][c]));
-                    *reinterpret_cast<uint4*>(O + o_byte(g + 8 * hh, a_local, 8 * (2 * q + e))) = pk;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int c = e + 2 * hh;
+                        const uint4 pk =
+                            make_uint4(pack_bf16x2(y3[0][c], y3[1][c]), pack_bf16x2(y3[2][c], y3[3][c]),
+                                       pack_bf16x2(y3[4][c], y3[5][c]), pack_bf16x2(y3[6][c], y3[7][c]));
+                        *reinterpret_cast<uint4*>(O + o_byte(g + 8 * hh, a_local, 8 * (2 * q + e))) = pk;
+                    }
                 }
+            } else {
+                // fp32 outputs back into E where this pencil's inputs were (beta = i2 + 8 i3)
+#pragma unroll
+                for (int l = 0; l < 8; ++l)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int beta = l + 8 * (2 * q + e);
+                            E[e_index<QB>(beta >> 5, g + 8 * hh, a_local, beta)] = y3[l][e + 2 * hh];
+                        }
             }
         }
         __syncthreads();
+        if constexpr (QB > 0) {
+            quant_row<QB>(E, reinterpret_cast<unsigned char*>(S), p, row0, r, warp, lane, qbar, qparity, remote_s,
+                          remote_qbar);
+            if constexpr (QB >= 64) qparity ^= 1;
+        }
         cluster_arrive();             // my E has been read: the partner may send the next tile
 
         prev_row0 = row0;             // its output is stored during the next tile's first task
     }
-    if (prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
+    if (QB == 0 && prev_row0 >= 0) store_row(O, p, prev_row0, warp, r, lane);
     cluster_wait();                   // matches the last arrive; no bulk copy is in flight
     tmem_fence_before_sync();
     __syncthreads();
@@ -608,6 +764,11 @@ bool is_d4096_radix8(const harp_plan_s* p) {
     return true;
 }
 
+// The variants: bf16 rows out, then int8 codes for quantizer blocks of 32, 64, 128, 256.
+const void* const kKernels[] = {(const void*)harp_fast_d4096_fwd_kernel<0>, (const void*)harp_fast_d4096_fwd_kernel<32>,
+                                (const void*)harp_fast_d4096_fwd_kernel<64>, (const void*)harp_fast_d4096_fwd_kernel<128>,
+                                (const void*)harp_fast_d4096_fwd_kernel<256>};
+
 // The coefficient table and the launch attributes of the specialized kernel, built once per
 // plan by materialization (on the materializing stream): afterwards launches only read
 // them, so calls on any number of streams may run at once.
@@ -621,18 +782,25 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
         cudaGetLastError();
     });
     if (!g_encode) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-    cudaError_t e = cudaFuncSetAttribute(harp_fast_d4096_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+    cudaError_t e = cudaSuccess;
+    for (const void* k : kKernels) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     int nclusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&nclusters, (void*)harp_fast_d4096_fwd_kernel, &cfg);
+    for (const void* k : kKernels) {   // the variants' limits (equal in practice: one CTA per SM)
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+        if (e != cudaSuccess) break;
+        nclusters = k == kKernels[0] ? n : std::min(nclusters, n);
+    }
     if (e != cudaSuccess || nclusters < 1) {
         cudaGetLastError();
         return harp_fail(HARP_ERR_CUDA, "no cluster of two fits on this device");
@@ -662,15 +830,11 @@ harp_status prepare(harp_plan_s* p, cudaStream_t stream) {
 
 }  // namespace
 
-harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
-                              int64_t ld_y, harp_dtype in_dtype, harp_dir dir, void* stream_,
-                              harp_dtype out_dtype) {
-    if (!is_d4096_radix8(p) || in_dtype != HARP_BF16 || out_dtype != HARP_BF16 || dir != HARP_FORWARD)
-        return HARP_ERR_UNSUPPORTED;
-    // TMA input boxes need 16-byte aligned rows; output runs are 16-byte stores
-    if (((uintptr_t)x & 15) || (ld_x & 7) || ((uintptr_t)y & 15) || (ld_y & 7)) return HARP_ERR_UNSUPPORTED;
-    if (rows < 32 || rows > 0x7fffffffll) return HARP_ERR_UNSUPPORTED;
-    cudaStream_t stream = (cudaStream_t)stream_;
+namespace {
+
+// Encodes the input map and launches variant QB (0: bf16 rows to fp.y; else the quantizer).
+harp_status launch_variant(harp_plan_s* p, const void* x, int64_t rows, int64_t ld_x, FastParams fp, int qb,
+                           cudaStream_t stream) {
     const FastState* fs = static_cast<const FastState*>(p->fast);
     if (!fs || !fs->ready) return HARP_ERR_UNSUPPORTED;   // no table: the plan was not eligible or it failed
     const int64_t ntiles = (rows + kTile - 1) / kTile;
@@ -695,18 +859,55 @@ harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t ro
     }
     if (cr != CUDA_SUCCESS) return harp_fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)cr));
 
-    FastParams fp;
-    fp.y = reinterpret_cast<__nv_bfloat16*>(y);
     fp.rows = rows;
-    fp.ldy = ld_y;
     fp.ntiles = (int)ntiles;
     fp.frag = reinterpret_cast<const float4*>(fs->frag);
     fp.status = p->d_status;
-    harp_fast_d4096_fwd_kernel<<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp);
+    switch (qb) {
+        case 0: harp_fast_d4096_fwd_kernel<0><<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp); break;
+        case 32: harp_fast_d4096_fwd_kernel<32><<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp); break;
+        case 64: harp_fast_d4096_fwd_kernel<64><<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp); break;
+        case 128: harp_fast_d4096_fwd_kernel<128><<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp); break;
+        case 256: harp_fast_d4096_fwd_kernel<256><<<2 * pairs, kThreads, kSmemBytes, stream>>>(tmap, fp); break;
+        default: return HARP_ERR_UNSUPPORTED;
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return harp_fail(HARP_ERR_CUDA, cudaGetErrorString(e));
     harp_set_last_kernel("harp_fast_d4096_fwd_kernel");
     return HARP_OK;
+}
+
+}  // namespace
+
+harp_status launch_apply_fast(harp_plan_s* p, const void* x, void* y, int64_t rows, int64_t ld_x,
+                              int64_t ld_y, harp_dtype in_dtype, harp_dir dir, void* stream,
+                              harp_dtype out_dtype) {
+    if (!is_d4096_radix8(p) || in_dtype != HARP_BF16 || out_dtype != HARP_BF16 || dir != HARP_FORWARD)
+        return HARP_ERR_UNSUPPORTED;
+    // TMA input boxes need 16-byte aligned rows; output runs are 16-byte stores
+    if (((uintptr_t)x & 15) || (ld_x & 7) || ((uintptr_t)y & 15) || (ld_y & 7)) return HARP_ERR_UNSUPPORTED;
+    if (rows < 32 || rows > 0x7fffffffll) return HARP_ERR_UNSUPPORTED;
+    FastParams fp = {};
+    fp.y = reinterpret_cast<__nv_bfloat16*>(y);
+    fp.ldy = ld_y;
+    return launch_variant(p, x, rows, ld_x, fp, 0, (cudaStream_t)stream);
+}
+
+harp_status launch_apply_fast_quant(harp_plan_s* p, const void* x, int64_t rows, int64_t ld_x, int8_t* q,
+                                    int64_t ld_q, float* scales, int64_t ld_s, int qblock, harp_dir dir,
+                                    void* stream) {
+    if (!is_d4096_radix8(p) || dir != HARP_FORWARD) return HARP_ERR_UNSUPPORTED;
+    if (qblock != 32 && qblock != 64 && qblock != 128 && qblock != 256) return HARP_ERR_UNSUPPORTED;
+    // TMA input boxes: 16-byte aligned rows; codes leave as 16-byte stores; scales as floats
+    if (((uintptr_t)x & 15) || (ld_x & 7) || ((uintptr_t)q & 15) || (ld_q & 15) || ((uintptr_t)scales & 3))
+        return HARP_ERR_UNSUPPORTED;
+    if (rows < 32 || rows > 0x7fffffffll) return HARP_ERR_UNSUPPORTED;
+    FastParams fp = {};
+    fp.q = q;
+    fp.ldq = ld_q;
+    fp.scales = scales;
+    fp.lds = ld_s;
+    return launch_variant(p, x, rows, ld_x, fp, qblock, (cudaStream_t)stream);
 }
 
 void fast_prepare(harp_plan_s* p, void* stream) {

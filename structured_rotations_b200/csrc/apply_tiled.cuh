@@ -286,10 +286,10 @@ __host__ __device__ __forceinline__ int stage_groups(int nb, int qv, int nthread
 
 // All items of one stage: items j = tid, tid + T, ...; item j is block c = j % nb of the
 // sub-tiles g = j / nb, g + G, ...  The block's coefficients are loaded into registers at
-// the start of the item (a second register buffer to prefetch the next block costs more
-// in register moves than it saves in latency at 8 warps per SM), except the first item's,
-// which the caller has already requested (prefetch_first) before the barrier that opens the
-// stage, so its L2 latency overlaps the barrier wait.
+// the start of the item (for radix 8 with 256 threads, one item ahead into a second register
+// block; elsewhere the registers are not there), except the first item's, which the caller has
+// already requested (prefetch_first) before the barrier that opens the stage, so its L2
+// latency overlaps the barrier wait.
 template <int B, bool INV, int V, int NT>
 __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, const FastDiv& nbd,
                                           const FastDiv& sdv, typename VecOf<V>::T* tile, int d, int qv,
@@ -306,24 +306,45 @@ __device__ __forceinline__ void run_stage(const float* __restrict__ sb, int s, c
     it.hi = sdv.div(it.c);
     it.lo = it.c - s * it.hi;
     const int dhi = sdv.div(NT), dlo = NT - s * dhi;
+    auto advance = [&](ItemPos& q) {
+        q.c += NT;
+        q.lo += dlo;
+        q.hi += dhi;
+        if (q.lo >= s) {
+            q.lo -= s;
+            ++q.hi;
+        }
+        if (q.c >= nb) {   // wrapped into the next sub-tile group (small nb only)
+            do {
+                q.c -= nb;
+                ++q.g;
+            } while (q.c >= nb);
+            q.hi = sdv.div(q.c);
+            q.lo = q.c - s * q.hi;
+        }
+    };
+    if constexpr (B == 8 && NT == 256) {
+        // Radix 8 with 256 threads (registers to spare): two register blocks take turns, so
+        // the next item's block is in flight while this item's FMAs run, with no moves.
+        float w1[64];
+        for (int j = tid; j < items; j += 2 * NT) {
+            ItemPos it1 = it;
+            advance(it1);
+            const bool has1 = j + NT < items;
+            if (has1) load_block<B>(w1, sb, it1.c);
+            apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, w);
+            ItemPos it2 = it1;
+            advance(it2);
+            if (j + 2 * NT < items) load_block<B>(w, sb, it2.c);
+            if (has1) apply_item<B, INV, V>(tile, d, qv, G, s, mask, it1, w1);
+            it = it2;
+        }
+        return;
+    }
     for (int j = tid; j < items; j += NT) {
         if (j != tid) load_block<B>(w, sb, it.c);   // the first item's block is already requested
         apply_item<B, INV, V>(tile, d, qv, G, s, mask, it, w);
-        it.c += NT;
-        it.lo += dlo;
-        it.hi += dhi;
-        if (it.lo >= s) {
-            it.lo -= s;
-            ++it.hi;
-        }
-        if (it.c >= nb) {   // wrapped into the next sub-tile group (small nb only)
-            do {
-                it.c -= nb;
-                ++it.g;
-            } while (it.c >= nb);
-            it.hi = sdv.div(it.c);
-            it.lo = it.c - s * it.hi;
-        }
+        advance(it);
     }
 }
 
@@ -707,8 +728,11 @@ __device__ __forceinline__ void drain_tile_quant(const typename VecOf<V>::T* til
 // CL = 1: one CTA holds whole rows.  CL = 2 (slab mode, schedules whose last radix is 2):
 // a cluster of two CTAs shares each tile, CTA r holding columns [r d/2, (r+1) d/2) of its
 // rows; stages 0..m-2 stay inside a slab, the last one is cross_stage.
-template <typename TIn, typename TOut, bool INV, int MASK, int V, int NT, int CL>
+// FUSED: a stage runs inside the fill or the drain (p.fuse_first / p.fuse_last); a kernel of its
+// own, so that the kernels without fused stages carry none of their code and registers.
+template <typename TIn, typename TOut, bool INV, int MASK, int V, int NT, int CL, bool FUSED>
 __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant__ TiledParams p) {
+    static_assert(!FUSED || (V == 4 && CL == 1 && NT == 256), "fused stages: whole rows, 4-row sub-tiles, 256 threads");
     extern __shared__ __align__(128) unsigned char smem[];
     using VT = typename VecOf<V>::T;
     const int d = (int)p.pd.d;
@@ -735,7 +759,7 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
     // block is requested before the barrier that precedes the stage
     float w[64];
     // stages fused into the fill / drain (4-row sub-tiles of whole rows only) are not run here
-    const bool fused = V == 4 && CL == 1 && NT == 256;   // the launcher fuses only with 256 threads
+    constexpr bool fused = FUSED;
     const int step0 = fused && p.fuse_first ? 1 : 0;
     const int step1 = m_local - (fused && p.fuse_last ? 1 : 0);
     const int t_first = INV ? m_local - 1 - step0 : step0;
@@ -743,7 +767,7 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
     // Without fused stages the first block is requested early (before the loop, and before the
     // drain of the previous tile), so its latency hides behind the drain and the fill; with them
     // it is requested after the fill, whose fused stage needs the registers.
-    const bool early = !(fused && (p.fuse_first || p.fuse_last));
+    constexpr bool early = !FUSED;
     if (early && step0 < step1)
         prefetch_first<MASK, V, NT>(p, t_first, (int)((min((int64_t)R, p.rows - t_idx * R) + V - 1) / V), dl, rank,
                                     w);
@@ -776,6 +800,12 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         const int nr = (int)min((int64_t)R, p.rows - row0);
         const int qv = (nr + V - 1) / V;
         const int n_staged = min(nr, p.staged_rows);
+        if constexpr (FUSED) {
+            // w's value from the last tile is dead (the first stage's block is requested after
+            // the fill): saying so leaves its registers to the fused fill and drain
+#pragma unroll
+            for (int k = 0; k < 64; ++k) w[k] = 0.f;
+        }
         if (n_staged && !failed) {
             bool ok = mbar_wait(bar, parity, p.wait_limit);
             if (__syncthreads_or(!ok)) {
@@ -792,7 +822,7 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
             }
             parity ^= 1;
         }
-        if constexpr (V == 4 && CL == 1 && NT == 256) {
+        if constexpr (FUSED) {
             if (p.fuse_first)
                 fill_tile_fused<NT, TIn, INV>((float4*)tile, dl, nr, n_staged, (const TIn*)stage_buf,
                                               (const TIn*)p.x + row0 * p.ld_x + col0, p.ld_x, p.fuse_first,
@@ -826,7 +856,7 @@ __global__ void __launch_bounds__(NT, 1) harp_tiled_kernel(const __grid_constant
         if constexpr (std::is_same<TOut, int8_t>::value)
             drain_tile_quant<V, NT>(tile, dl, nr, (int8_t*)p.y + row0 * p.ld_y, p.ld_y, p.mask,
                                     p.scales + row0 * p.ld_s, p.ld_s, p.qlanes);
-        else if constexpr (V == 4 && CL == 1 && NT == 256) {
+        else if constexpr (FUSED) {
             if (p.fuse_last)
                 drain_tile_fused<NT, TOut, INV>((const float4*)tile, dl, nr, (TOut*)p.y + row0 * p.ld_y + col0,
                                                 p.ld_y, p.fuse_last, sb_of(INV ? 0 : m_local - 1));
@@ -857,15 +887,15 @@ constexpr int kThreadChoices[] = {256, 384};
 // Slab-mode kernels exist for the radix sets that contain 2.
 constexpr bool has_slab_kernel(int mask) { return ((mask >> 2) & 1) != 0 && mask != 0x1fc; }
 
-template <typename TIn, typename TOut, bool INV, int V, int NT, int CL, int I>
+template <typename TIn, typename TOut, bool INV, int V, int NT, int CL, int I, bool FUSED = false>
 cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
     if constexpr (I < kNumMasks) {
-        if (which != I) return launch_mask<TIn, TOut, INV, V, NT, CL, I + 1>(which, tp, smem, grid, stream);
+        if (which != I) return launch_mask<TIn, TOut, INV, V, NT, CL, I + 1, FUSED>(which, tp, smem, grid, stream);
         if constexpr ((V == 1 && !has_row_major_kernel(kMasks[I])) ||
                       (CL == 2 && (V != 4 || !has_slab_kernel(kMasks[I]) || std::is_same<TOut, int8_t>::value))) {
             return cudaErrorInvalidValue;
         } else {
-            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT, CL>;
+            auto kern = harp_tiled_kernel<TIn, TOut, INV, kMasks[I], V, NT, CL, FUSED>;
             cudaError_t e = (cudaError_t)harp_set_smem_limit((const void*)kern, (int)smem);
             if (e != cudaSuccess) return e;
             if constexpr (CL == 1) {
@@ -895,6 +925,12 @@ cudaError_t launch_mask(int which, const TiledParams& tp, size_t smem, int grid,
 
 template <typename TIn, typename TOut, bool INV, int V>
 cudaError_t launch_nt(int which, int nt, int cl, const TiledParams& tp, size_t smem, int grid, cudaStream_t stream) {
+    if constexpr (V == 4) {
+        if (tp.fuse_first || tp.fuse_last) {
+            if (nt != 256 || cl != 1) return cudaErrorInvalidValue;
+            return launch_mask<TIn, TOut, INV, 4, 256, 1, 0, true>(which, tp, smem, grid, stream);
+        }
+    }
     if (cl == 2) {
         if (nt == 384) return launch_mask<TIn, TOut, INV, V, 384, 2, 0>(which, tp, smem, grid, stream);
         return launch_mask<TIn, TOut, INV, V, 256, 2, 0>(which, tp, smem, grid, stream);

@@ -113,6 +113,11 @@ harp_status launch_apply_cluster(const harp_plan_s* p, const void* x, void* y, i
 // `stream` for plans it covers; a no-op for other plans.  Called by materialization, so
 // every later launch only reads the table.  A plan whose table cannot be built (no
 // cluster fits, no tensor-map encoder) is left without one and runs on the other kernels.
+// The specialized kernel with the blockwise quantizer as its epilogue (harp_apply_quant on a
+// d = 4096 (8,8,8,8) plan, forward); HARP_ERR_UNSUPPORTED for anything else.
+harp_status launch_apply_fast_quant(harp_plan_s* p, const void* x, int64_t rows, int64_t ld_x, int8_t* q,
+                                    int64_t ld_q, float* scales, int64_t ld_s, int qblock, harp_dir dir,
+                                    void* stream);
 void fast_prepare(harp_plan_s* p, void* stream);
 void host_io_free(harp_plan_s* p);
 

@@ -50,9 +50,52 @@ def test_quant_vs_oracle(name, direction, rows, qblock):
     xe = W.draw_encoded(W.get(name), 0, rows)
     q, s = gp.apply_quant(to_dev(xe), qblock, direction)
     torch.cuda.synchronize()
-    assert H.last_kernel() == "harp_tiled_kernel"
+    # d = 4096 forward takes the specialized kernel's quantizing variant
+    fast = name == "d4096" and direction == "forward"
+    assert H.last_kernel() == ("harp_fast_d4096_fwd_kernel" if fast else "harp_tiled_kernel")
     x64 = decode(xe)
     _check(q.cpu().numpy(), s.cpu().numpy(), tr.apply(x64, direction), x64, qblock, f"{name} {direction} {rows}")
+
+
+@pytest.mark.parametrize("qblock", [32, 64, 128, 256])
+@pytest.mark.parametrize("rows", [32, 45, 1000])
+def test_fast_kernel_quantizer_vs_oracle(monkeypatch, rows, qblock):
+    """d = 4096 (8,8,8,8) forward on the specialized kernel: each CTA of a pair holds half of
+    every quantizer block of 64 coordinates or more (its 32 pencils), so the block maxima are
+    exchanged between the two; a zero row (scale 0, codes 0), a one-hot row and ragged last
+    tiles included."""
+    monkeypatch.setenv("HARP_KERNEL", "fast")
+    gp, tr = plans("d4096")
+    xe = W.draw_encoded(W.get("d4096"), 0, rows)
+    xe[3] = 0
+    xe[7] = 0
+    xe[7, 1234] = W.encode_bf16(np.array([5.0]))[0]
+    q, s = gp.apply_quant(to_dev(xe), qblock)
+    torch.cuda.synchronize()
+    assert H.last_kernel() == "harp_fast_d4096_fwd_kernel"
+    x64 = decode(xe)
+    qh, sh = q.cpu().numpy(), s.cpu().numpy()
+    _check(qh, sh, tr.forward(x64), x64, qblock, f"fast rows={rows} qblock={qblock}")
+    assert np.all(qh[3] == 0) and np.all(sh[3] == 0)
+    gp.device_status()
+
+
+def test_fast_kernel_quantizer_padded_outputs(monkeypatch):
+    """Padded code and scale rows: the kernel writes exactly rows x 4096 codes and
+    rows x 4096 / qblock scales."""
+    monkeypatch.setenv("HARP_KERNEL", "fast")
+    gp, tr = plans("d4096")
+    rows = 77
+    xe = W.draw_encoded(W.get("d4096"), 0, rows)
+    qp = torch.full((rows, 4096 + 48), 5, dtype=torch.int8, device=DEV)
+    sp = torch.full((rows, 40), -1.0, device=DEV)
+    gp.apply_quant(to_dev(xe), 128, q=qp[:, :4096], scales=sp[:, :32])
+    torch.cuda.synchronize()
+    assert H.last_kernel() == "harp_fast_d4096_fwd_kernel"
+    x64 = decode(xe)
+    _check(qp[:, :4096].cpu().numpy(), sp[:, :32].cpu().numpy(), tr.forward(x64), x64, 128, "fast padded")
+    assert torch.all(qp[:, 4096:] == 5) and torch.all(sp[:, 32:] == -1.0)
+    gp.device_status()
 
 
 def test_quant_full_size_on_sampled_rows():
