@@ -180,12 +180,18 @@ def test_two_sided_small_full_compare():
 
 
 def test_two_sided_full_size_sampled_rows():
+    """C4 at full size (28672 x 8192): 448 output rows against the oracle, one in every 64-row
+    slab (the column kernel's second pass) with the offsets inside the slab running through all
+    64 residues seven times (so every 448-row set {p + 64 v} of its first pass is hit), plus the
+    first and last rows."""
     w = W.get("two_sided")
     pu, tu, pv, tv = _two_sided_plans(w.u_schedule, w.schedule, w)
     wt = W.draw_encoded(w, 0, w.n_out, w.n_in)
     out = to_host(H.apply_two_sided(pu, pv, to_dev(wt)))
     torch.cuda.synchronize()
-    rows = W.sample_rows(w.n_out, 6)
+    k = np.arange(w.n_out // 64)
+    rows = np.unique(np.concatenate([64 * k + (k % 64), W.sample_rows(w.n_out, 6)]))
+    assert np.unique(rows // 64).size == w.n_out // 64 and np.unique(rows % 64).size == 64
     # row i of T_U^T W T_V is (T_U e_i)^T W T_V
     e = np.zeros((rows.size, w.n_out))
     e[np.arange(rows.size), rows] = 1.0
