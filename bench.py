@@ -61,6 +61,10 @@ def parse_args():
     ap.add_argument("--grad-rows", type=int, default=0,
                     help="time only the calibration backward (harp_grad_theta) on this many d=4096 rows and "
                          "print its line (for profiling that kernel alone)")
+    ap.add_argument("--two-sided-cols", type=int, default=0,
+                    help="time only the two-sided rotation T_U^T W T_V of the two-sided workload with W cut to "
+                         "this many columns (8^k, 2 * 8^k or 4 * 8^k; V = (8,...,8, 2 or 4), the workload's own "
+                         "schedule at 8192) and print one JSON line")
     ap.add_argument("--decode-rows", type=int, default=0,
                     help="time only decode-shaped calls (this many rows of the d=8192 int8 workload, forward) "
                          "and print their line (for profiling that call alone)")
@@ -436,30 +440,7 @@ def side_measurements(args, H, W, torch, device, peak):
                         "hbm_frac": (rb + coef) / (dev_us / 1e6) / 1e9 / peak})
         del xd, yd
     del pd_
-    # two-sided: W_out = T_U^T W T_V, V on the rows (d = n_in), U on the columns (d = n_out)
-    w4 = W.get("two_sided")
-    th_v = W.draw_theta(H.theta_count(w4.schedule), w4.theta_sigma, w4.theta_seed)
-    th_u = W.draw_theta(H.theta_count(w4.u_schedule), w4.theta_sigma, w4.theta_seed + 7)
-    pv = H.Plan(w4.n_in, w4.schedule, theta=th_v, sign_seed=w4.sign_seed).materialize()
-    pu = H.Plan(w4.n_out, w4.u_schedule, theta=th_u, sign_seed=w4.sign_seed + 11).materialize()
-    wt = to_device_bf16(W.draw_encoded(w4, 0, w4.n_out, w4.n_in), torch, device)
-    wo = torch.empty_like(wt)
-    ws = torch.empty(H.workspace_bytes(w4.n_out, w4.n_in), dtype=torch.uint8, device=device)
-    for _ in range(2):
-        H.apply_two_sided(pu, pv, wt, wo, ws)
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    st = 3
-    e0.record(stream)
-    for _ in range(st):
-        H.apply_two_sided(pu, pv, wt, wo, ws)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / st
-    b4 = 2 * (2 * w4.n_out * w4.n_in * 2)        # two passes, each reading and writing W once
-    out.append({"workload": WORKLOAD_TEXT["two_sided"], "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9,
-                "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak, "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"})
+    out.append(two_sided_measurement(args, H, W, torch, device, peak))
     out.append(fit_measurement(H, W, torch, device, peak, pv, wo, w4))
     del wt, wo, ws
     out.append(quant_measurement(args, H, W, torch, device, peak))
@@ -573,6 +554,49 @@ def compose_measurement(args, H, W, torch, device, peak):
             "two_passes_ms": two, "two_passes_kernels": "harp_fast_d4096_fwd_kernel x 2 (bf16 between)"}
 
 
+
+def two_sided_measurement(args, H, W, torch, device, peak, n_in=None):
+    """The two-sided weight rotation W_out = T_U^T W T_V on the two-sided workload (V on the
+    rows, d = n_in; U on the columns, d = n_out); n_in cuts W to fewer columns, with V's
+    schedule the workload's (8,8,8,8,2) shortened to match (a smaller case for profiles).
+    Algorithmic HBM bytes: two passes, each reading and writing W once."""
+    import numpy as np
+    w4 = W.get("two_sided")
+    v_sched = tuple(w4.schedule)
+    if n_in and n_in != w4.n_in:
+        k = 0
+        while 8 ** (k + 1) <= n_in:
+            k += 1
+        r = n_in // 8 ** k
+        if k < 1 or r * 8 ** k != n_in or r not in (1, 2, 4):
+            raise SystemExit(f"--two-sided-cols must be 8^k, 2 * 8^k or 4 * 8^k, got {n_in}")
+        v_sched = (8,) * k + ((r,) if r > 1 else ())
+    n_in = int(np.prod(v_sched))
+    th_v = W.draw_theta(H.theta_count(v_sched), w4.theta_sigma, w4.theta_seed)
+    th_u = W.draw_theta(H.theta_count(w4.u_schedule), w4.theta_sigma, w4.theta_seed + 7)
+    pv = H.Plan(n_in, v_sched, theta=th_v, sign_seed=w4.sign_seed).materialize()
+    pu = H.Plan(w4.n_out, w4.u_schedule, theta=th_u, sign_seed=w4.sign_seed + 11).materialize()
+    wt = to_device_bf16(W.draw_encoded(w4, 0, w4.n_out, n_in), torch, device)
+    wo = torch.empty_like(wt)
+    ws = torch.empty(H.workspace_bytes(w4.n_out, n_in), dtype=torch.uint8, device=device)
+    for _ in range(2):
+        H.apply_two_sided(pu, pv, wt, wo, ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st = 3
+    e0.record(stream)
+    for _ in range(st):
+        H.apply_two_sided(pu, pv, wt, wo, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / st
+    b4 = 2 * (2 * w4.n_out * n_in * 2)        # two passes, each reading and writing W once
+    text = WORKLOAD_TEXT["two_sided"] if n_in == w4.n_in else \
+        f"two-sided T_U^T W T_V: W {w4.n_out}x{n_in} bf16, U {tuple(w4.u_schedule)}, V {v_sched}"
+    return {"workload": text, "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9, "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak,
+            "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"}
+
 def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):
     """The fused rotate-then-quantize pass (harp_apply_quant) on the d = 4096 workload:
     bf16 rows in, int8 codes and one fp32 scale per 128 coordinates out; algorithmic HBM
@@ -683,6 +707,9 @@ def run_ours(args):
         print(json.dumps({"workload": f"d=8192 schedule (8,8,8,8,2), int8 theta, {args.decode_rows} bf16 rows, "
                                       "forward", "device_us_per_call": dev_us, "host_us_per_call": host_us,
                           "us_per_call": wall_us, "kernel": kn}))
+        return 0
+    if args.two_sided_cols:
+        print(json.dumps(two_sided_measurement(args, H, W, torch, device, peaks()[0], args.two_sided_cols)))
         return 0
     if args.quant_rows:
         peak, _ = peaks()
