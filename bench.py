@@ -440,9 +440,10 @@ def side_measurements(args, H, W, torch, device, peak):
                         "hbm_frac": (rb + coef) / (dev_us / 1e6) / 1e9 / peak})
         del xd, yd
     del pd_
-    out.append(two_sided_measurement(args, H, W, torch, device, peak))
-    out.append(fit_measurement(H, W, torch, device, peak, pv, wo, w4))
-    del wt, wo, ws
+    ts, pv, wo = two_sided_measurement(args, H, W, torch, device, peak, keep=True)
+    out.append(ts)
+    out.append(fit_measurement(H, W, torch, device, peak, pv, wo, W.get("two_sided")))
+    del pv, wo
     out.append(quant_measurement(args, H, W, torch, device, peak))
     out.append(compose_measurement(args, H, W, torch, device, peak))
     out.append(moment_measurement(args, H, W, torch, device, peak))
@@ -555,11 +556,12 @@ def compose_measurement(args, H, W, torch, device, peak):
 
 
 
-def two_sided_measurement(args, H, W, torch, device, peak, n_in=None):
+def two_sided_measurement(args, H, W, torch, device, peak, n_in=None, keep=False):
     """The two-sided weight rotation W_out = T_U^T W T_V on the two-sided workload (V on the
     rows, d = n_in; U on the columns, d = n_out); n_in cuts W to fewer columns, with V's
     schedule the workload's (8,8,8,8,2) shortened to match (a smaller case for profiles).
-    Algorithmic HBM bytes: two passes, each reading and writing W once."""
+    Algorithmic HBM bytes: two passes, each reading and writing W once.  keep: also return
+    plan V and the rotated weight (the fit terms' line uses them)."""
     import numpy as np
     w4 = W.get("two_sided")
     v_sched = tuple(w4.schedule)
@@ -594,8 +596,10 @@ def two_sided_measurement(args, H, W, torch, device, peak, n_in=None):
     b4 = 2 * (2 * w4.n_out * n_in * 2)        # two passes, each reading and writing W once
     text = WORKLOAD_TEXT["two_sided"] if n_in == w4.n_in else \
         f"two-sided T_U^T W T_V: W {w4.n_out}x{n_in} bf16, U {tuple(w4.u_schedule)}, V {v_sched}"
-    return {"workload": text, "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9, "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak,
-            "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"}
+    res = {"workload": text, "ms": ms, "hbm_gbs": b4 / (ms / 1e3) / 1e9, "hbm_frac": b4 / (ms / 1e3) / 1e9 / peak,
+           "kernel": "harp_apply_two_sided: harp_tiled_kernel (rows) + 2 x harp_cols_kernel (columns)"}
+    del wt, ws
+    return (res, pv, wo) if keep else res
 
 def quant_measurement(args, H, W, torch, device, peak, qblock=128, rows=None):
     """The fused rotate-then-quantize pass (harp_apply_quant) on the d = 4096 workload:
