@@ -556,6 +556,20 @@ def compose_measurement(args, H, W, torch, device, peak):
 
 
 
+def two_sided_v_schedule(n_in, w4):
+    """V's schedule for a two-sided case with n_in columns: the workload's own at its n_in (or
+    when n_in is 0), else radix 8 stages and one radix 2 or 4 (n_in = 8^k, 2 8^k or 4 8^k)."""
+    if not n_in or n_in == w4.n_in:
+        return tuple(w4.schedule)
+    k = 0
+    while 8 ** (k + 1) <= n_in:
+        k += 1
+    r = n_in // 8 ** k
+    if k < 1 or r * 8 ** k != n_in or r not in (1, 2, 4):
+        raise SystemExit(f"--two-sided-cols must be 8^k, 2 * 8^k or 4 * 8^k, got {n_in}")
+    return (8,) * k + ((r,) if r > 1 else ())
+
+
 def two_sided_measurement(args, H, W, torch, device, peak, n_in=None, keep=False):
     """The two-sided weight rotation W_out = T_U^T W T_V on the two-sided workload (V on the
     rows, d = n_in; U on the columns, d = n_out); n_in cuts W to fewer columns, with V's
@@ -564,15 +578,7 @@ def two_sided_measurement(args, H, W, torch, device, peak, n_in=None, keep=False
     plan V and the rotated weight (the fit terms' line uses them)."""
     import numpy as np
     w4 = W.get("two_sided")
-    v_sched = tuple(w4.schedule)
-    if n_in and n_in != w4.n_in:
-        k = 0
-        while 8 ** (k + 1) <= n_in:
-            k += 1
-        r = n_in // 8 ** k
-        if k < 1 or r * 8 ** k != n_in or r not in (1, 2, 4):
-            raise SystemExit(f"--two-sided-cols must be 8^k, 2 * 8^k or 4 * 8^k, got {n_in}")
-        v_sched = (8,) * k + ((r,) if r > 1 else ())
+    v_sched = two_sided_v_schedule(n_in, w4)
     n_in = int(np.prod(v_sched))
     th_v = W.draw_theta(H.theta_count(v_sched), w4.theta_sigma, w4.theta_seed)
     th_u = W.draw_theta(H.theta_count(w4.u_schedule), w4.theta_sigma, w4.theta_seed + 7)

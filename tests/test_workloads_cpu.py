@@ -30,3 +30,18 @@ def test_upstream_gradients_are_standard_normal_and_not_the_rows():
 def test_empty_draws():
     w = W.get("d64")
     assert W.draw_upstream(w, 5, 0).shape == (0, 64)
+
+
+def test_two_sided_cases_of_the_bench():
+    """The bench's smaller two-sided cases (--two-sided-cols): V's schedule multiplies out to
+    the column count, the full size keeps the workload's own schedule, others are refused."""
+    import bench
+    w4 = W.get("two_sided")
+    assert bench.two_sided_v_schedule(0, w4) == tuple(w4.schedule)
+    assert bench.two_sided_v_schedule(w4.n_in, w4) == tuple(w4.schedule)
+    for n, want in ((1024, (8, 8, 8, 2)), (2048, (8, 8, 8, 4)), (512, (8, 8, 8)), (64, (8, 8))):
+        assert bench.two_sided_v_schedule(n, w4) == want
+        assert int(np.prod(want)) == n
+    for bad in (3000, 24, 12, 4):
+        with pytest.raises(SystemExit):
+            bench.two_sided_v_schedule(bad, w4)
